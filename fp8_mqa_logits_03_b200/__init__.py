@@ -1,1 +1,226 @@
-"""B200-native fp8 MQA indexer (logits + top-k)."""
+"""B200-native fp8 MQA indexer: logits + top-k over fp8 keys.
+
+A thin Python binding over the C ABI of ``libfp8idx.so`` (``include/fp8idx.h``):
+each function only checks and marshals torch CUDA tensors into pointers and
+sizes and calls the entry point of the same name on the current CUDA stream.
+Every arithmetic step runs in the library's CUDA kernels; there is no CPU or
+PyTorch fallback, and a missing or unloadable library raises.
+
+  mqa_logits(q, k, s, w, ks, ke)                         -> logits [m, n] f32
+  topk_rows(logits, ks, ke, topk)                        -> idx [m, topk] i32
+  mqa_logits_topk(q, k, s, w, ks, ke, topk)              -> idx (and values)
+  paged_mqa_logits_topk(q, k_pages, s_pages, w, block_table, seq_lens, R, topk)
+
+q/k are fp8 e4m3fn bytes (torch.uint8 or torch.float8_e4m3fn), s/w float32,
+ks/ke/block_table/seq_lens int32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import workloads  # noqa: F401  (seeded synthetic inputs)
+
+H = 32
+D = 128
+MAX_TOPK = 2048
+PAGE_SIZE = 64
+
+OK, EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA = 0, 1, 2, 3, 4
+STATUS_WAIT_TIMEOUT, STATUS_BAD_PAGE, STATUS_SEQ_TOO_LONG = 1, 2, 4
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8idx.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class Fp8IdxError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"fp8idx error {code}: {msg}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m fp8_mqa_logits_03_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+            L.fp8idx_mqa_logits.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i32, i32, vp, i64, vp]
+            L.fp8idx_topk_rows.argtypes = [vp, i64, vp, vp, i64, i64, i32, vp, vp]
+            L.fp8idx_mqa_logits_topk_workspace.argtypes = [i64, i64, i32, i32, i32]
+            L.fp8idx_mqa_logits_topk_workspace.restype = sz
+            L.fp8idx_mqa_logits_topk.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i32, i32, i32,
+                                                 vp, vp, vp, sz, vp]
+            L.fp8idx_paged_mqa_logits_topk_workspace.argtypes = [i64, i32, i32, i32, i32, i32]
+            L.fp8idx_paged_mqa_logits_topk_workspace.restype = sz
+            L.fp8idx_paged_mqa_logits_topk.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i64,
+                                                       i32, i32, i32, i32, vp, vp, vp, sz, vp]
+            L.fp8idx_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
+            L.fp8idx_last_error.restype = ctypes.c_char_p
+            L.fp8idx_num_sms.restype = ctypes.c_int
+            L.fp8idx_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+            for name in ("fp8idx_mqa_logits", "fp8idx_topk_rows", "fp8idx_mqa_logits_topk",
+                         "fp8idx_paged_mqa_logits_topk", "fp8idx_read_device_status"):
+                getattr(L, name).restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise Fp8IdxError(rc, lib().fp8idx_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _bytes(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    if t.dtype != torch.uint8:
+        raise TypeError(f"{name} must be fp8 e4m3fn bytes (uint8 or float8_e4m3fn), got {t.dtype}")
+    return _dev(t, name)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def num_sms() -> int:
+    return lib().fp8idx_num_sms()
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    lib().fp8idx_set_wait_limit_ns(int(ns))
+
+
+def read_device_status(workspace=None, stream=None) -> int:
+    v = ctypes.c_int(0)
+    _check(lib().fp8idx_read_device_status(_ptr(workspace), ctypes.byref(v), _stream(stream)))
+    return v.value
+
+
+# ---------------------------------------------------------------------------- calls
+
+def mqa_logits(q, k, s, w, ks, ke, logits=None, stream=None) -> torch.Tensor:
+    """fp32 logits [m, n]: s[j] * sum_h w[i,h] * ReLU(q[i,h].k[j]) on [ks, ke), -inf elsewhere."""
+    q = _bytes(q, "q")
+    k = _bytes(k, "k")
+    s = _dev(s, "s", torch.float32)
+    w = _dev(w, "w", torch.float32)
+    ks = _dev(ks, "ks", torch.int32)
+    ke = _dev(ke, "ke", torch.int32)
+    m, n = q.shape[0], k.shape[0]
+    if logits is None:
+        logits = torch.empty((m, n), dtype=torch.float32, device=q.device)
+    if logits.dim() != 2 or logits.stride(1) != 1 or logits.dtype != torch.float32:
+        raise ValueError("logits must be a [m, >=n] float32 tensor with unit column stride")
+    _check(lib().fp8idx_mqa_logits(_ptr(q), _ptr(k), _ptr(s), _ptr(w), _ptr(ks), _ptr(ke), m, n,
+                                   q.shape[1], q.shape[2], _ptr(logits), logits.stride(0),
+                                   _stream(stream)))
+    return logits
+
+
+def topk_rows(logits, ks, ke, topk: int = MAX_TOPK, out=None, n=None, stream=None) -> torch.Tensor:
+    """Top-k column indices of each logit row over [ks, ke) (ties: lower index), -1 padded."""
+    logits = _dev(logits, "logits", torch.float32) if logits.stride(1) == 1 else None
+    if logits is None:
+        raise ValueError("logits must have unit column stride")
+    ks = _dev(ks, "ks", torch.int32)
+    ke = _dev(ke, "ke", torch.int32)
+    m = logits.shape[0]
+    n = logits.shape[1] if n is None else n
+    if out is None:
+        out = torch.empty((m, topk), dtype=torch.int32, device=logits.device)
+    _check(lib().fp8idx_topk_rows(_ptr(logits), logits.stride(0), _ptr(ks), _ptr(ke), m, n, topk,
+                                  _ptr(out), _stream(stream)))
+    return out
+
+
+def mqa_logits_topk_workspace_size(m: int, n: int, topk: int = MAX_TOPK) -> int:
+    return int(lib().fp8idx_mqa_logits_topk_workspace(m, n, H, D, topk))
+
+
+def paged_workspace_size(B: int, R: int, max_blocks: int, topk: int = MAX_TOPK) -> int:
+    return int(lib().fp8idx_paged_mqa_logits_topk_workspace(B, R, max_blocks, H, D, topk))
+
+
+def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A 256-byte aligned device buffer (torch's caching allocator aligns to 512)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8,
+                       device=device if device is not None else "cuda")
+
+
+def mqa_logits_topk(q, k, s, w, ks, ke, topk: int = MAX_TOPK, out=None, out_vals=None,
+                    workspace=None, return_values: bool = False, stream=None):
+    """Fused logits + top-k without materialising the m x n logits."""
+    q = _bytes(q, "q")
+    k = _bytes(k, "k")
+    s = _dev(s, "s", torch.float32)
+    w = _dev(w, "w", torch.float32)
+    ks = _dev(ks, "ks", torch.int32)
+    ke = _dev(ke, "ke", torch.int32)
+    m, n = q.shape[0], k.shape[0]
+    if out is None:
+        out = torch.empty((m, topk), dtype=torch.int32, device=q.device)
+    if return_values and out_vals is None:
+        out_vals = torch.empty((m, topk), dtype=torch.float32, device=q.device)
+    need = mqa_logits_topk_workspace_size(m, n, topk)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    _check(lib().fp8idx_mqa_logits_topk(_ptr(q), _ptr(k), _ptr(s), _ptr(w), _ptr(ks), _ptr(ke), m,
+                                        n, q.shape[1], q.shape[2], topk, _ptr(out), _ptr(out_vals),
+                                        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return (out, out_vals) if return_values else out
+
+
+def paged_mqa_logits_topk(q, k_pages, s_pages, w, block_table, seq_lens, R: int,
+                          topk: int = MAX_TOPK, out=None, out_vals=None, workspace=None,
+                          return_values: bool = False, stream=None):
+    """Paged decode/verify: R rows per request, keys through a 64-token block table."""
+    q = _bytes(q, "q")
+    k_pages = _bytes(k_pages, "k_pages")
+    s_pages = _dev(s_pages, "s_pages", torch.float32)
+    w = _dev(w, "w", torch.float32)
+    block_table = _dev(block_table, "block_table", torch.int32)
+    seq_lens = _dev(seq_lens, "seq_lens", torch.int32)
+    B, max_blocks = block_table.shape
+    num_pages = k_pages.shape[0]
+    page_size = k_pages.shape[1]
+    rows = q.shape[0]
+    if rows != B * R:
+        raise ValueError(f"q has {rows} rows, expected B*R = {B * R}")
+    if out is None:
+        out = torch.empty((rows, topk), dtype=torch.int32, device=q.device)
+    if return_values and out_vals is None:
+        out_vals = torch.empty((rows, topk), dtype=torch.float32, device=q.device)
+    need = paged_workspace_size(B, R, max_blocks, topk)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    _check(lib().fp8idx_paged_mqa_logits_topk(_ptr(q), _ptr(k_pages), _ptr(s_pages), _ptr(w),
+                                              _ptr(block_table), _ptr(seq_lens), B, R, max_blocks,
+                                              num_pages, page_size, q.shape[1], q.shape[2], topk,
+                                              _ptr(out), _ptr(out_vals), _ptr(workspace),
+                                              workspace.numel(), _stream(stream)))
+    return (out, out_vals) if return_values else out

@@ -1,0 +1,435 @@
+// api.cu -- the C ABI (include/fp8idx.h): argument checks, workspace plans,
+// TMA descriptor encoding and kernel launches.  Host code only.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/fp8idx.h"
+#include "kernels.cuh"
+
+namespace fp8idx {
+__device__ int g_logits_status;  // device status of the last fp8idx_mqa_logits call
+}
+
+namespace {
+
+using namespace fp8idx;
+
+thread_local std::string t_last_error;
+unsigned long long g_wait_limit_ns = 2000000000ull;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return code;
+}
+
+int ok() {
+  t_last_error.clear();
+  return FP8IDX_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(FP8IDX_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// A [rows, 128]-byte matrix read in boxes of [box_rows, 128] with the
+// 128-byte swizzle the MMA descriptors expect.  Rows past the end read as 0.
+int make_rows128_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(FP8IDX_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDim)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kDim), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FP8IDX_ECUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return FP8IDX_OK;
+}
+
+// ---------------------------------------------------------------- plans
+
+struct Plan {
+  int R = 8;
+  int n_chunks = 1;
+  int chunk_keys = 0;
+  int num_units = 0;
+  int grid = 0;
+  int cap = 0;
+  size_t off_cand = 0, off_part = 0, off_cnt = 0, total = 0;
+};
+
+int candidate_capacity(int topk) { return static_cast<int>(round_up(4 * topk + 256, 128)); }
+
+void finish_plan(Plan& pl, int64_t groups, int sms, int topk) {
+  pl.num_units = static_cast<int>(groups * pl.n_chunks);
+  pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(pl.num_units, sms)));
+  pl.cap = candidate_capacity(topk);
+  size_t off = kStatusBytes;
+  pl.off_cand = off;
+  off += round_up(static_cast<int64_t>(sms) * pl.R * pl.cap * 8, 256);
+  if (pl.n_chunks > 1) {
+    pl.off_part = off;
+    off += round_up(static_cast<int64_t>(pl.num_units) * pl.R * topk * 8, 256);
+    pl.off_cnt = off;
+    off += round_up(static_cast<int64_t>(pl.num_units) * pl.R * 4, 256);
+  }
+  pl.total = off;
+}
+
+// Row blocks of 8 rows; when they cannot fill the GPU, the key axis is cut
+// into chunks so that about two units land on every SM.
+Plan plan_prefill(int64_t m, int64_t n, int topk, int sms) {
+  Plan pl;
+  pl.R = 8;
+  const int64_t groups = ceil_div(m, pl.R);
+  const int64_t axis = std::max<int64_t>(n, 1);
+  pl.chunk_keys = static_cast<int>(round_up(axis, kBlockKeys));
+  pl.n_chunks = 1;
+  if (groups < sms) {
+    const int64_t want = ceil_div(2 * static_cast<int64_t>(sms), groups);
+    const int64_t ck = round_up(ceil_div(axis, want), kBlockKeys);
+    pl.chunk_keys = static_cast<int>(ck);
+    pl.n_chunks = static_cast<int>(ceil_div(axis, ck));
+  }
+  finish_plan(pl, groups, sms, topk);
+  return pl;
+}
+
+// One unit per (request, key chunk); chunks sized so that about four units
+// land on every SM (context lengths differ, so many chunks are short or empty).
+Plan plan_paged(int64_t B, int R, int max_blocks, int topk, int sms) {
+  Plan pl;
+  pl.R = R;
+  const int64_t axis = static_cast<int64_t>(max_blocks) * kPageSize;
+  pl.chunk_keys = static_cast<int>(round_up(axis, kBlockKeys));
+  pl.n_chunks = 1;
+  if (B < 4 * static_cast<int64_t>(sms)) {
+    const int64_t want = ceil_div(4 * static_cast<int64_t>(sms), B);
+    const int64_t ck = round_up(ceil_div(axis, want), kBlockKeys);
+    pl.chunk_keys = static_cast<int>(ck);
+    pl.n_chunks = static_cast<int>(ceil_div(axis, ck));
+  }
+  finish_plan(pl, B, sms, topk);
+  return pl;
+}
+
+int check_shape(int H, int D) {
+  if (H != kHeads || D != kDim)
+    return fail(FP8IDX_EUNSUPPORTED, "only H=32, D=128 are supported (got H=%d, D=%d)", H, D);
+  return FP8IDX_OK;
+}
+
+int check_topk(int topk) {
+  if (topk < 1 || topk > kMaxTopK)
+    return fail(FP8IDX_EINVAL, "topk must be in [1, %d] (got %d)", kMaxTopK, topk);
+  return FP8IDX_OK;
+}
+
+#define FP8IDX_TRY(x)          \
+  do {                         \
+    int _rc = (x);             \
+    if (_rc != FP8IDX_OK) return _rc; \
+  } while (0)
+
+int check_prefill_inputs(const uint8_t* q, const uint8_t* k, const float* s, const float* w,
+                         const int32_t* ks, const int32_t* ke, int64_t m, int64_t n) {
+  if (m < 0 || n < 0) return fail(FP8IDX_EINVAL, "negative size (m=%lld, n=%lld)", (long long)m, (long long)n);
+  if (m > (int64_t(1) << 25)) return fail(FP8IDX_EINVAL, "m=%lld is too large", (long long)m);
+  if (n >= (int64_t(1) << 31) - kBlockKeys) return fail(FP8IDX_EINVAL, "n=%lld is too large", (long long)n);
+  if (m == 0) return FP8IDX_OK;
+  if (!q || !w || !ks || !ke) return fail(FP8IDX_EINVAL, "null q, w, ks or ke");
+  if (n > 0 && (!k || !s)) return fail(FP8IDX_EINVAL, "null k or s");
+  if (!aligned(q, 16) || (k && !aligned(k, 16)))
+    return fail(FP8IDX_EINVAL, "q and k must be 16-byte aligned");
+  if (!aligned(s, 4) || !aligned(w, 4) || !aligned(ks, 4) || !aligned(ke, 4))
+    return fail(FP8IDX_EINVAL, "s, w, ks and ke must be 4-byte aligned");
+  return FP8IDX_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+const char* fp8idx_last_error(void) { return t_last_error.c_str(); }
+
+int fp8idx_num_sms(void) { return device_sms(); }
+
+void fp8idx_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
+
+int fp8idx_mqa_logits(const uint8_t* q, const uint8_t* k, const float* s, const float* w,
+                      const int32_t* ks, const int32_t* ke, int64_t m, int64_t n, int H, int D,
+                      float* logits, int64_t ld_logits, void* stream) {
+  FP8IDX_TRY(check_shape(H, D));
+  FP8IDX_TRY(check_prefill_inputs(q, k, s, w, ks, ke, m, n));
+  if (m == 0 || n == 0) return ok();
+  if (!logits || !aligned(logits, 4)) return fail(FP8IDX_EINVAL, "logits must be non-null and 4-byte aligned");
+  if (ld_logits < n) return fail(FP8IDX_EINVAL, "ld_logits (%lld) < n (%lld)", (long long)ld_logits, (long long)n);
+  const int sms = device_sms();
+  if (sms <= 0) return fail(FP8IDX_ECUDA, "no CUDA device");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // One unit per 8-row block; small m splits the key axis (each unit writes
+  // its own column range, so no merge is needed).
+  Plan pl = plan_prefill(m, n, 1, sms);
+  IndexerParams p;
+  memset(&p, 0, sizeof(p));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, m * kHeads, pl.R * kHeads));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_k, k, n, kBlockKeys));
+  p.s = s;
+  p.w = w;
+  p.ks = ks;
+  p.ke = ke;
+  p.n = n;
+  p.m = static_cast<int>(m);
+  p.topk = 1;
+  p.n_chunks = pl.n_chunks;
+  p.chunk_keys = pl.chunk_keys;
+  p.num_units = pl.num_units;
+  p.logits = logits;
+  p.ld_logits = ld_logits;
+  int* status = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_logits_status);
+  if (e != cudaSuccess) return cuda_fail(e, "status symbol");
+  e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+  p.status = status;
+  p.wait_limit_ns = g_wait_limit_ns;
+  e = launch_indexer_prefill_logits(p, pl.grid, st);
+  if (e != cudaSuccess) return cuda_fail(e, "mqa_logits launch");
+  return ok();
+}
+
+int fp8idx_topk_rows(const float* logits, int64_t ld, const int32_t* ks, const int32_t* ke,
+                     int64_t m, int64_t n, int topk, int32_t* out, void* stream) {
+  FP8IDX_TRY(check_topk(topk));
+  if (m < 0 || n < 0) return fail(FP8IDX_EINVAL, "negative size");
+  if (m > INT32_MAX || n >= (int64_t(1) << 31)) return fail(FP8IDX_EINVAL, "size too large");
+  if (m == 0) return ok();
+  if (!ks || !ke || !out || (n > 0 && !logits)) return fail(FP8IDX_EINVAL, "null pointer");
+  if (!aligned(logits, 4) || !aligned(ks, 4) || !aligned(ke, 4) || !aligned(out, 4))
+    return fail(FP8IDX_EINVAL, "pointers must be 4-byte aligned");
+  if (ld < n) return fail(FP8IDX_EINVAL, "ld (%lld) < n (%lld)", (long long)ld, (long long)n);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  TopkRowsParams p{logits, ld, ks, ke, n, static_cast<int>(m), topk, out};
+  cudaError_t e = launch_topk_rows(p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "topk_rows launch");
+  return ok();
+}
+
+size_t fp8idx_mqa_logits_topk_workspace(int64_t m, int64_t n, int H, int D, int topk) {
+  if (H != kHeads || D != kDim || topk < 1 || topk > kMaxTopK || m < 0 || n < 0) return 0;
+  const int sms = device_sms();
+  if (sms <= 0) return 0;
+  return plan_prefill(std::max<int64_t>(m, 1), n, topk, sms).total;
+}
+
+int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, const float* w,
+                           const int32_t* ks, const int32_t* ke, int64_t m, int64_t n, int H,
+                           int D, int topk, int32_t* out_idx, float* out_vals, void* ws,
+                           size_t ws_bytes, void* stream) {
+  FP8IDX_TRY(check_shape(H, D));
+  FP8IDX_TRY(check_topk(topk));
+  FP8IDX_TRY(check_prefill_inputs(q, k, s, w, ks, ke, m, n));
+  if (m == 0) return ok();
+  if (!out_idx || !aligned(out_idx, 4) || !aligned(out_vals, 4))
+    return fail(FP8IDX_EINVAL, "out_idx must be non-null; outputs 4-byte aligned");
+  const int sms = device_sms();
+  if (sms <= 0) return fail(FP8IDX_ECUDA, "no CUDA device");
+  Plan pl = plan_prefill(m, n, topk, sms);
+  if (!ws || !aligned(ws, 256)) return fail(FP8IDX_EINVAL, "workspace must be non-null and 256-byte aligned");
+  if (ws_bytes < pl.total)
+    return fail(FP8IDX_EWORKSPACE, "workspace too small (%zu < %zu bytes)", ws_bytes, pl.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+  if (n == 0) {
+    e = launch_fill_empty(out_idx, out_vals, static_cast<int>(m), topk, st);
+    if (e != cudaSuccess) return cuda_fail(e, "fill launch");
+    return ok();
+  }
+  IndexerParams p;
+  memset(&p, 0, sizeof(p));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, m * kHeads, pl.R * kHeads));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_k, k, n, kBlockKeys));
+  p.s = s;
+  p.w = w;
+  p.ks = ks;
+  p.ke = ke;
+  p.n = n;
+  p.m = static_cast<int>(m);
+  p.topk = topk;
+  p.n_chunks = pl.n_chunks;
+  p.chunk_keys = pl.chunk_keys;
+  p.num_units = pl.num_units;
+  p.out_idx = out_idx;
+  p.out_vals = out_vals;
+  p.status = reinterpret_cast<int*>(wsb);
+  p.cand = reinterpret_cast<uint2*>(wsb + pl.off_cand);
+  p.cand_cap = pl.cap;
+  if (pl.n_chunks > 1) {
+    p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
+    p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
+  }
+  p.wait_limit_ns = g_wait_limit_ns;
+  e = launch_indexer_prefill_topk(p, pl.grid, st);
+  if (e != cudaSuccess) return cuda_fail(e, "mqa_logits_topk launch");
+  if (pl.n_chunks > 1) {
+    MergeParams mp{p.part, p.part_cnt, static_cast<int>(m), pl.R, pl.n_chunks, topk, out_idx, out_vals};
+    e = launch_merge(mp, st);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  }
+  return ok();
+}
+
+size_t fp8idx_paged_mqa_logits_topk_workspace(int64_t B, int R, int max_blocks, int H, int D,
+                                              int topk) {
+  if (H != kHeads || D != kDim || topk < 1 || topk > kMaxTopK || B < 0 || max_blocks < 1 ||
+      (R != 4 && R != 8))
+    return 0;
+  const int sms = device_sms();
+  if (sms <= 0) return 0;
+  return plan_paged(std::max<int64_t>(B, 1), R, max_blocks, topk, sms).total;
+}
+
+int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const float* s_pages,
+                                 const float* w, const int32_t* block_table,
+                                 const int32_t* seq_lens, int64_t B, int R, int max_blocks,
+                                 int64_t num_pages, int page_size, int H, int D, int topk,
+                                 int32_t* out_idx, float* out_vals, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  FP8IDX_TRY(check_shape(H, D));
+  FP8IDX_TRY(check_topk(topk));
+  if (page_size != kPageSize) return fail(FP8IDX_EUNSUPPORTED, "page_size must be 64 (got %d)", page_size);
+  if (R != 4 && R != 8) return fail(FP8IDX_EUNSUPPORTED, "rows per request must be 4 or 8 (got %d)", R);
+  if (B < 0 || num_pages < 0 || max_blocks < 1) return fail(FP8IDX_EINVAL, "bad sizes");
+  if (B * R > (int64_t(1) << 25)) return fail(FP8IDX_EINVAL, "too many rows");
+  if (static_cast<int64_t>(max_blocks) * kPageSize >= (int64_t(1) << 31) - kBlockKeys ||
+      num_pages * kPageSize >= (int64_t(1) << 31))
+    return fail(FP8IDX_EINVAL, "paged key space too large");
+  if (B == 0) return ok();
+  if (!q || !w || !block_table || !seq_lens || !out_idx)
+    return fail(FP8IDX_EINVAL, "null q, w, block_table, seq_lens or out_idx");
+  if (num_pages > 0 && (!k_pages || !s_pages)) return fail(FP8IDX_EINVAL, "null k_pages or s_pages");
+  if (!aligned(q, 16) || !aligned(k_pages, 16))
+    return fail(FP8IDX_EINVAL, "q and k_pages must be 16-byte aligned");
+  if (!aligned(s_pages, 4) || !aligned(w, 4) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
+      !aligned(out_idx, 4) || !aligned(out_vals, 4))
+    return fail(FP8IDX_EINVAL, "pointers must be 4-byte aligned");
+  const int sms = device_sms();
+  if (sms <= 0) return fail(FP8IDX_ECUDA, "no CUDA device");
+  Plan pl = plan_paged(B, R, max_blocks, topk, sms);
+  if (!ws || !aligned(ws, 256)) return fail(FP8IDX_EINVAL, "workspace must be non-null and 256-byte aligned");
+  if (ws_bytes < pl.total)
+    return fail(FP8IDX_EWORKSPACE, "workspace too small (%zu < %zu bytes)", ws_bytes, pl.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+  if (num_pages == 0) {
+    e = launch_fill_empty(out_idx, out_vals, static_cast<int>(B * R), topk, st);
+    if (e != cudaSuccess) return cuda_fail(e, "fill launch");
+    return ok();
+  }
+  IndexerParams p;
+  memset(&p, 0, sizeof(p));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, B * R * kHeads, R * kHeads));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_k, k_pages, num_pages * kPageSize, kPageSize));
+  p.s = s_pages;
+  p.w = w;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.m = static_cast<int>(B * R);
+  p.max_blocks = max_blocks;
+  p.num_pages = static_cast<int>(num_pages);
+  p.topk = topk;
+  p.n_chunks = pl.n_chunks;
+  p.chunk_keys = pl.chunk_keys;
+  p.num_units = pl.num_units;
+  p.out_idx = out_idx;
+  p.out_vals = out_vals;
+  p.status = reinterpret_cast<int*>(wsb);
+  p.cand = reinterpret_cast<uint2*>(wsb + pl.off_cand);
+  p.cand_cap = pl.cap;
+  if (pl.n_chunks > 1) {
+    p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
+    p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
+  }
+  p.wait_limit_ns = g_wait_limit_ns;
+  e = launch_indexer_paged_topk(p, R, pl.grid, st);
+  if (e != cudaSuccess) return cuda_fail(e, "paged_mqa_logits_topk launch");
+  if (pl.n_chunks > 1) {
+    MergeParams mp{p.part, p.part_cnt, static_cast<int>(B * R), pl.R, pl.n_chunks, topk, out_idx, out_vals};
+    e = launch_merge(mp, st);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  }
+  return ok();
+}
+
+int fp8idx_read_device_status(const void* ws, int* status_out, void* stream) {
+  if (!status_out) return fail(FP8IDX_EINVAL, "null status_out");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const void* src = ws;
+  if (!src) {
+    void* sym = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&sym, g_logits_status);
+    if (e != cudaSuccess) return cuda_fail(e, "status symbol");
+    src = sym;
+  }
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, src, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  *status_out = v;
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,88 @@
+// kernels.cuh -- parameter blocks and launch helpers shared by the kernels
+// and the C-ABI layer.  Host and device.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace fp8idx {
+
+constexpr int kHeads = 32;         // index heads
+constexpr int kDim = 128;          // index head dim (bytes per fp8 row)
+constexpr int kBlockKeys = 128;    // keys per tile = MMA M = TMEM lanes
+constexpr int kPageSize = 64;      // tokens per key page (paged form)
+constexpr int kMaxTopK = 2048;
+constexpr int kThreads = 320;      // 10 warps: TMA, MMA, 8 epilogue
+constexpr int kStatusBytes = 256;  // device status block at the head of every workspace
+
+// device status bits (workspace word 0)
+constexpr int kStatusWaitTimeout = 1;
+constexpr int kStatusBadPage = 2;
+constexpr int kStatusSeqLenTooLong = 4;
+
+enum Mode : int { kModeLogits = 0, kModeTopK = 1 };
+
+struct IndexerParams {
+  CUtensorMap tmap_q;  // q viewed as [rows * 32, 128] bytes, box {128, R * 32}
+  CUtensorMap tmap_k;  // keys [n, 128] (box {128, 128}) or pages [P * 64, 128] (box {128, 64})
+  const float* s;      // key scales [n] or [P * 64]
+  const float* w;      // head weights [m, 32]
+  const int32_t* ks;   // prefill ranges
+  const int32_t* ke;
+  const int32_t* block_table;  // paged: [B, max_blocks]
+  const int32_t* seq_lens;     // paged: [B]
+  int64_t n;                   // prefill: number of keys
+  int m;                       // query rows (prefill m, paged B * R)
+  int max_blocks;
+  int num_pages;
+  int topk;
+  int n_chunks;     // key chunks per row block / request
+  int chunk_keys;   // keys per chunk (multiple of 128)
+  int num_units;    // row blocks (or requests) x n_chunks
+  // logits mode
+  float* logits;
+  int64_t ld_logits;
+  // top-k outputs (direct mode: n_chunks == 1)
+  int32_t* out_idx;
+  float* out_vals;
+  // workspace
+  int* status;
+  uint2* cand;      // [gridDim.x][R][cand_cap] (order key, index)
+  int cand_cap;
+  uint2* part;      // split mode: [num_units][R][topk]
+  int* part_cnt;    // split mode: [num_units][R]
+  unsigned long long wait_limit_ns;
+};
+
+struct MergeParams {
+  const uint2* part;
+  const int* part_cnt;
+  int rows;          // total query rows
+  int R;             // rows per unit
+  int n_chunks;
+  int topk;
+  int32_t* out_idx;
+  float* out_vals;
+};
+
+struct TopkRowsParams {
+  const float* logits;
+  int64_t ld;
+  const int32_t* ks;
+  const int32_t* ke;
+  int64_t n;
+  int m;
+  int topk;
+  int32_t* out_idx;
+};
+
+// Launchers (kernels.cu).  They only enqueue work; validation is the caller's.
+cudaError_t launch_indexer_prefill_logits(const IndexerParams& p, int grid, cudaStream_t st);
+cudaError_t launch_indexer_prefill_topk(const IndexerParams& p, int grid, cudaStream_t st);
+cudaError_t launch_indexer_paged_topk(const IndexerParams& p, int R, int grid, cudaStream_t st);
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t st);
+cudaError_t launch_topk_rows(const TopkRowsParams& p, cudaStream_t st);
+cudaError_t launch_fill_empty(int32_t* out_idx, float* out_vals, int rows, int topk,
+                              cudaStream_t st);
+
+}  // namespace fp8idx

@@ -1,0 +1,155 @@
+/*
+ * fp8idx.h -- C ABI of the B200 (sm_100a) fp8 MQA indexer library.
+ *
+ * The operation (the sparse-attention indexer of the
+ * "bench_mqa_logits_chunking.py" page: module docstring, `_build` and
+ * `_run_chunked`, which call `deep_gemm.fp8_mqa_logits(q, (kv, kv_scales),
+ * weights, ks, ke)` and then `fast_topk_transform_fused(score, lengths, ...,
+ * topk, row_starts)`; GLM-5.1 shapes index_n_heads = 32, index_head_dim =
+ * 128, index_topk = 2048):
+ *
+ *   logits[i,j] = s[j] * sum_{h<H} w[i,h] * max(0, sum_{d<D} q[i,h,d] * k[j,d])
+ *                 for max(ks[i],0) <= j < min(ke[i],n), and -inf otherwise;
+ *   out[i,:]    = the k key indices of row i with the largest logits, ties
+ *                 going to the lower index, padded with -1 when fewer than
+ *                 k keys are valid.  The order inside a row is unspecified.
+ *
+ * q and k are fp8 e4m3fn bytes (the "e4m3fn" format named on the
+ * "Serve GLM-5.3-Flash on SM80" page, commit notes); s and w are fp32; ks
+ * and ke are int32.  H must be 32 and D must be 128.
+ *
+ * Conventions shared by every call:
+ *   - All data pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates, frees, synchronises the stream or reads device data on
+ *     the host (except fp8idx_read_device_status, which is for tests).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only enqueues work on it and returns.
+ *   - Layouts are dense row-major: q [m, H, D], k [n, D], s [n], w [m, H],
+ *     ks/ke [m], out [m, topk].
+ *   - Alignment: q, k and k_pages 16 bytes (TMA); everything else 4 bytes;
+ *     workspaces 256 bytes.
+ *   - Errors are reported before anything is launched and leave the outputs
+ *     untouched: FP8IDX_EINVAL (null pointer, misalignment, negative size,
+ *     topk outside [1, 2048], ld_logits < n), FP8IDX_EUNSUPPORTED (H != 32,
+ *     D != 128, page_size != 64, rows_per_request not 4 or 8),
+ *     FP8IDX_EWORKSPACE (workspace smaller than the *_workspace() size),
+ *     FP8IDX_ECUDA (a CUDA call failed; see fp8idx_last_error()).
+ *     m == 0 (or B == 0) is a no-op returning FP8IDX_OK.
+ *   - Device-side problems that the host cannot see (a block-table entry
+ *     outside [0, num_pages), a sequence length beyond max_blocks * 64, a
+ *     pipeline wait that timed out) set bits in a status word at the head
+ *     of the workspace; read it with fp8idx_read_device_status().
+ *   - fp8 inputs holding NaN bytes (0x7F / 0xFF) give unspecified output.
+ */
+#ifndef FP8IDX_H_
+#define FP8IDX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  FP8IDX_OK = 0,
+  FP8IDX_EINVAL = 1,
+  FP8IDX_EUNSUPPORTED = 2,
+  FP8IDX_EWORKSPACE = 3,
+  FP8IDX_ECUDA = 4
+};
+
+/* device status bits (fp8idx_read_device_status) */
+enum {
+  FP8IDX_STATUS_WAIT_TIMEOUT = 1,   /* a pipeline wait gave up; outputs are invalid      */
+  FP8IDX_STATUS_BAD_PAGE = 2,       /* a block-table entry outside [0, num_pages)        */
+  FP8IDX_STATUS_SEQ_TOO_LONG = 4    /* seq_lens[b] > max_blocks * page_size (clamped)    */
+};
+
+/*
+ * Materialised logits (the `fp8_mqa_logits` call of the
+ * "bench_mqa_logits_chunking.py" page, `_run_chunked`), except that every
+ * entry outside [ks[i], ke[i]) is written as -inf.
+ *   q       [m, H, D] e4m3 bytes          k  [n, D] e4m3 bytes
+ *   s       [n] fp32 key scales           w  [m, H] fp32 head weights
+ *   ks, ke  [m] int32 (clamped to [0, n] on the device)
+ *   logits  [m, ld_logits] fp32 output; columns [0, n) of every row are
+ *           written, ld_logits >= n.  Needs m * ld_logits * 4 bytes: callers
+ *           with large m * n chunk the rows (one call per row chunk, passing
+ *           offset q, w, ks, ke and logits pointers).
+ * No workspace.  Device status of this call: fp8idx_read_device_status(NULL, ...).
+ */
+int fp8idx_mqa_logits(const uint8_t* q, const uint8_t* k, const float* s, const float* w,
+                      const int32_t* ks, const int32_t* ke, int64_t m, int64_t n, int H, int D,
+                      float* logits, int64_t ld_logits, void* stream);
+
+/*
+ * Top-k of materialised logit rows (the `fast_topk_transform_fused(score,
+ * lengths, ..., topk, row_starts)` call of the same page with the identity
+ * page table): for each row i, the topk largest logits[i, j] over
+ * max(ks[i],0) <= j < min(ke[i],n), ties to the lower j, padded with -1.
+ *   logits [m, ld] fp32; ks, ke [m] int32; out [m, topk] int32.
+ * No workspace.
+ */
+int fp8idx_topk_rows(const float* logits, int64_t ld, const int32_t* ks, const int32_t* ke,
+                     int64_t m, int64_t n, int topk, int32_t* out, void* stream);
+
+/*
+ * Fused logits + top-k: the same result as fp8idx_mqa_logits followed by
+ * fp8idx_topk_rows, computed by streaming over 128-key tiles without ever
+ * holding the m x n logits.  Arguments as above; out_idx [m, topk] int32;
+ * out_vals [m, topk] fp32 receives the matching logits (-inf padding) and
+ * may be NULL.  ws / ws_bytes: caller-owned device workspace of at least
+ * fp8idx_mqa_logits_topk_workspace(m, n, H, D, topk) bytes, 256-byte
+ * aligned, reused freely between calls on the same stream (calls that may
+ * overlap on the device need separate workspaces).  The size depends on the
+ * current device's SM count.
+ */
+size_t fp8idx_mqa_logits_topk_workspace(int64_t m, int64_t n, int H, int D, int topk);
+int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, const float* w,
+                           const int32_t* ks, const int32_t* ke, int64_t m, int64_t n, int H,
+                           int D, int topk, int32_t* out_idx, float* out_vals, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * Paged decode / verify form (the paged MQA logits named on the
+ * "Serve GLM-5.3-Flash on SM80" page, commit notes): B requests with R query
+ * rows each (MTP width R).  Key j of request b is slot j % 64 of physical
+ * page block_table[b * max_blocks + j / 64]; row t of request b (global row
+ * b * R + t) sees keys [0, seq_lens[b] - R + t + 1), clamped to
+ * [0, seq_lens[b]].  Output indices are logical token positions.
+ *   q           [B * R, H, D] e4m3 bytes     w        [B * R, H] fp32
+ *   k_pages     [num_pages, 64, D] e4m3       s_pages  [num_pages, 64] fp32
+ *   block_table [B, max_blocks] int32 (entries past a request's pages are
+ *               never read)                   seq_lens [B] int32
+ *   out_idx     [B * R, topk] int32           out_vals [B * R, topk] fp32 or NULL
+ * R must be 4 or 8; page_size must be 64.
+ */
+size_t fp8idx_paged_mqa_logits_topk_workspace(int64_t B, int R, int max_blocks, int H, int D,
+                                              int topk);
+int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const float* s_pages,
+                                 const float* w, const int32_t* block_table,
+                                 const int32_t* seq_lens, int64_t B, int R, int max_blocks,
+                                 int64_t num_pages, int page_size, int H, int D, int topk,
+                                 int32_t* out_idx, float* out_vals, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/*
+ * Tests and diagnostics.  fp8idx_read_device_status synchronises `stream`
+ * and copies the status word written by the last call that used workspace
+ * `ws` (ws == NULL: the last fp8idx_mqa_logits call) into *status_out.
+ */
+int fp8idx_read_device_status(const void* ws, int* status_out, void* stream);
+/* Message for the last non-OK return on this thread ("" if none). */
+const char* fp8idx_last_error(void);
+/* Number of SMs of the current device (what the workspace sizes assume). */
+int fp8idx_num_sms(void);
+/* Upper bound in nanoseconds on any single pipeline wait inside a kernel
+ * (default 2e9).  Tests lower it to exercise the timeout path. */
+void fp8idx_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8IDX_H_ */
