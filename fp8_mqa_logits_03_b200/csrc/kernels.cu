@@ -379,6 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
             int64_t e = U.len - R + rl + 1;
             hi_r[r] = max(min(e, U.len), static_cast<int64_t>(0));
           }
+          // a unit only owns the keys of its chunk (its last tile may overhang)
+          lo_r[r] = max(lo_r[r], U.cbeg);
+          hi_r[r] = min(hi_r[r], U.cend);
         }
       }
       if (tid_wg < RW * kHeads) {
