@@ -1,0 +1,400 @@
+#!/usr/bin/env python3
+"""Benchmark: fused fp8 MQA logits + top-2048 on the causal-prefill workload.
+
+One step = one pass of the whole indexer hot path over the workload
+m = 8192 query rows x n = 35000 keys (H = 32, D = 128, ks = 0,
+ke[i] = n - m + i + 1, top-k = 2048): range resolution, TMA staging,
+tcgen05 fp8 contraction, fused ReLU / head-weight / scale / mask epilogue,
+streaming top-k filter and exact per-row select, in one persistent kernel.
+
+Prints ONE JSON line (rank 0).  `value` is algorithmic TFLOP/s over all
+ranks: 8192 flop (2 * H * D) per valid (row, key) pair, divided by the max
+over ranks of the device time of K steps.  Inputs are resident in HBM;
+L2 is flushed (a 256 MiB write) before every timed step.  `e2e` is the same
+metric through the same C-ABI call with the inputs copied from pinned host
+memory and the top-k indices copied back inside each timed step.
+
+--impl reference times the float64 CPU oracle instead, on a bounded sample
+of the same workload's rows per step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fp8_mqa_logits_03_b200 import workloads  # noqa: E402
+
+WORKLOAD = 1
+METRIC = "indexer fp8 TFLOP/s & rows·keys/s (fused logits+top-2048), % of roofline"
+UNIT = "TFLOP/s"
+FLOP_PER_PAIR = 2 * workloads.H * workloads.D  # 8192
+
+
+def strict_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, allow_abbrev=False)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, choices=sorted(workloads.WORKLOADS), default=WORKLOAD,
+                    help="workload index (default 1, the headline causal prefill)")
+    ap.add_argument("--quick", action="store_true",
+                    help="device timing only: skip the end-to-end pass and the CPU baseline")
+    a = ap.parse_args(argv)
+    if a.gpus < 1 or a.steps < 1 or a.warmup < 3:
+        ap.error("need --gpus >= 1, --steps >= 1, --warmup >= 3")
+    return a
+
+
+def valid_pairs(ks: torch.Tensor, ke: torch.Tensor, n: int) -> int:
+    lo = ks.long().clamp(min=0)
+    hi = torch.maximum(lo, ke.long().clamp(max=n))
+    return int((hi - lo).sum())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p.get("hbm_gbs", 6650.0)), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # pragma: no cover - no NVML
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def dist_setup(gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != gpus:
+        raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local, pg
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+def max_over_ranks(pg, x: float) -> float:
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world, pg):
+    import oracle
+    if rank != 0:
+        return None
+    d = workloads.make_workload(WORKLOAD)
+    q, k, s, w = (d[x].numpy() for x in ("q", "k", "s", "w"))
+    ks, ke = d["ks"].numpy(), d["ke"].numpy()
+    m, n = d["m"], d["n"]
+    per_step = 4  # rows per step, walked through the workload with a fixed stride
+    order = (np.arange(m, dtype=np.int64) * 2459) % m
+    threads = oracle.host_threads()
+
+    def step(i):
+        rows = order[(i * per_step) % m: (i * per_step) % m + per_step]
+        oracle.mqa_logits_topk_rows(q, k, s, w, ks, ke, workloads.TOPK, rows=rows, threads=threads)
+        return sum(max(0, min(int(ke[r]), n) - max(int(ks[r]), 0)) for r in rows)
+
+    for i in range(args.warmup):
+        step(i)
+    pairs = 0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        pairs += step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = FLOP_PER_PAIR * pairs / dt / 1e12
+    sample = (f"{args.steps} steps x {per_step} query rows of {d['name']} "
+              f"({pairs} valid (row, key) pairs), float64 logits + full-sort top-2048")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": d["name"], "m": m, "n": n, "H": workloads.H, "D": workloads.D,
+                   "topk": workloads.TOPK, "seed": d["seed"]},
+        "rows_keys_per_s": pairs / dt,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def cpu_baseline(d, budget_s: float = 12.0):
+    """The oracle as it stands on this host's cores, on a strided row sample."""
+    import oracle
+    q, k, s, w = (d[x].numpy() for x in ("q", "k", "s", "w"))
+    ks, ke = d["ks"].numpy(), d["ke"].numpy()
+    m, n = d["m"], d["n"]
+    threads = oracle.host_threads()
+    order = (np.arange(m, dtype=np.int64) * 2459) % m
+    batch = max(threads, 16)
+    pairs, done, t0 = 0, 0, time.perf_counter()
+    while done < m and time.perf_counter() - t0 < budget_s:
+        rows = order[done: done + batch]
+        oracle.mqa_logits_topk_rows(q, k, s, w, ks, ke, workloads.TOPK, rows=rows, threads=threads)
+        pairs += sum(max(0, min(int(ke[r]), n) - max(int(ks[r]), 0)) for r in rows)
+        done += len(rows)
+    dt = time.perf_counter() - t0
+    return {"value": FLOP_PER_PAIR * pairs / dt / 1e12, "unit": UNIT, "cores": threads,
+            "kind": "oracle",
+            "sample": f"{done} of {m} query rows of {d['name']} (strided), {pairs} valid pairs, "
+                      f"{dt:.1f} s wall, float64 logits + full-sort top-2048"}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def make_case(fx, index, dev):
+    """Device-resident inputs, outputs, workspace and the C-ABI call for one workload."""
+    d = workloads.make_workload(index)
+    topk = workloads.TOPK
+    if index == 4:
+        keys = ("q", "k_pages", "s_pages", "w", "block_table", "seq_lens")
+        host = {x: d[x].pin_memory() for x in keys}
+        dv = {x: host[x].to(dev) for x in keys}
+        rows, R = d["B"] * d["R"], d["R"]
+        out = torch.empty((rows, topk), dtype=torch.int32, device=dev)
+        ws = fx.alloc_workspace(fx.paged_workspace_size(d["B"], R, d["max_blocks"], topk), dev)
+        L = d["seq_lens"].long()
+        ke = torch.stack([(L - R + t + 1).clamp(min=0) for t in range(R)], 1).clamp(max=L[:, None])
+        pairs = int(ke.sum())
+        # algorithmic bytes: every key row + scale read once per request, the block-table
+        # entries in use, q and w of the request's rows, and the top-k written
+        nbytes = int((L * (workloads.D + 4)).sum() + ((L + 63) // 64).sum() * 4
+                     + rows * (workloads.H * workloads.D + workloads.H * 4 + topk * 4))
+
+        def call():
+            fx.paged_mqa_logits_topk(**dv, R=R, topk=topk, out=out, workspace=ws)
+        kernel = "indexer_kernel<4,true,1> (paged fused logits + top-k) + merge_kernel"
+        bound = "hbm"
+    else:
+        keys = ("q", "k", "s", "w", "ks", "ke")
+        host = {x: d[x].pin_memory() for x in keys}
+        dv = {x: host[x].to(dev) for x in keys}
+        out = torch.empty((d["m"], topk), dtype=torch.int32, device=dev)
+        ws = fx.alloc_workspace(fx.mqa_logits_topk_workspace_size(d["m"], d["n"], topk), dev)
+        pairs = valid_pairs(d["ks"], d["ke"], d["n"])
+        nbytes = int(d["m"] * (workloads.H * workloads.D + workloads.H * 4 + 8 + topk * 4)
+                     + d["n"] * (workloads.D + 4))
+
+        def call():
+            fx.mqa_logits_topk(**dv, topk=topk, out=out, workspace=ws)
+        kernel = "indexer_kernel<8,false,1> (fused logits + top-k)"
+        bound = "tensor"
+    out_host = torch.empty(out.shape, dtype=torch.int32).pin_memory()
+    return dict(d=d, call=call, host=host, dv=dv, out=out, out_host=out_host, ws=ws, pairs=pairs,
+                flops=FLOP_PER_PAIR * pairs, bytes=nbytes, kernel=kernel, bound=bound)
+
+
+def run_ours(args, rank, world, local, pg):
+    import fp8_mqa_logits_03_b200 as fx
+    from fp8_mqa_logits_03_b200 import build
+    if rank == 0 or not os.path.exists(fx.LIB_PATH):
+        build.build()
+    barrier(pg)
+    fx.lib()
+    dev = torch.device("cuda", local)
+    case = make_case(fx, args.workload, dev)  # every rank: one independent slice of this shape
+    d, call, host, dv, out, out_host, ws = (case[x] for x in
+                                            ("d", "call", "host", "dv", "out", "out_host", "ws"))
+    pairs, flops = case["pairs"], case["flops"]
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    assert fx.read_device_status(ws) == 0, "device status set during warm-up"
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(pg)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            call()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(pg)
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total_ms = max_over_ranks(pg, sum(step_ms))
+    ms_per_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    status = fx.read_device_status(ws)
+    kstats = fx.read_device_stats(ws)  # counters of the last timed call
+
+    # end to end through the same call: pinned H2D of the inputs, D2H of the top-k
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    e2e_value = e2e_ms = None
+    if not args.quick:
+        e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier(pg)
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.zero_()
+            e_starts[i].record(stream)
+            for x in host:
+                dv[x].copy_(host[x], non_blocking=True)
+            call()
+            out_host.copy_(out, non_blocking=True)
+            e_ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(pg)
+        e2e_ms = max_over_ranks(pg, sum(a.elapsed_time(b) for a, b in zip(e_starts, e_ends)))
+        e2e_value = world * flops * args.steps / (e2e_ms / 1e3) / 1e12
+
+    if rank != 0:
+        return None
+    bf16_peak, hbm_peak, peak_src = load_peaks()
+    fp8_peak = 2.0 * bf16_peak  # measured bf16 burst x nominal fp8/bf16 ratio (4.5 / 2.25)
+    mean_s = statistics.mean(step_ms) / 1e3
+    if case["bound"] == "tensor":
+        achieved = flops / mean_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp8_peak, "traffic": None,
+                "peak_source": f"{peak_src} bf16 burst {bf16_peak} TFLOP/s x 2 (fp8/bf16 nominal ratio)"}
+    else:
+        achieved = case["bytes"] / mean_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": None,
+                "peak_source": f"{peak_src} HBM copy bandwidth", "algorithmic_bytes": case["bytes"]}
+    roof["kernel"] = case["kernel"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3", "data": "synthetic",
+        "config": {"workload": d["name"], "H": workloads.H, "D": workloads.D, "topk": workloads.TOPK,
+                   "seed": d["seed"], "valid_pairs": pairs,
+                   "l2": "flushed before every timed step (256 MiB write, untimed)",
+                   "parallelism": f"replicas x{world} (one independent slice per GPU)"},
+        "rows_keys_per_s": world * pairs * args.steps / (total_ms / 1e3),
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "ms_per_step": None if e2e_ms is None else e2e_ms / args.steps},
+        "gpu_launches": args.steps * (2 if args.workload in (0, 4) else 1),
+        "clocks": clocks.summary(),
+        "device_status": status,
+        "kernel_stats": kstats,
+        "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)},
+    }
+    for key in ("m", "n", "B", "R"):
+        if key in d:
+            line["config"][key] = d[key]
+    if args.workload != 4 and not args.quick:
+        line["cpu_baseline"] = cpu_baseline(d)
+    return line
+
+
+def main():
+    args = strict_args()
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        if args.workload != WORKLOAD:
+            raise SystemExit("--impl reference times the headline workload only")
+        line = run_reference(args, 0, args.gpus, None)
+        print(json.dumps(line), flush=True)
+        return
+    rank, world, local, pg = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world, pg)
+        else:
+            line = run_ours(args, rank, world, local, pg)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
             L.fp8idx_paged_mqa_logits_topk.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i64,
                                                        i32, i32, i32, i32, vp, vp, vp, sz, vp]
             L.fp8idx_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
+            L.fp8idx_read_device_stats.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), i32, vp]
+            L.fp8idx_read_device_stats.restype = ctypes.c_int
             L.fp8idx_last_error.restype = ctypes.c_char_p
             L.fp8idx_num_sms.restype = ctypes.c_int
             L.fp8idx_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
@@ -119,6 +121,14 @@ def read_device_status(workspace=None, stream=None) -> int:
     v = ctypes.c_int(0)
     _check(lib().fp8idx_read_device_status(_ptr(workspace), ctypes.byref(v), _stream(stream)))
     return v.value
+
+
+def read_device_stats(workspace, stream=None) -> dict:
+    """Counters the fused top-k left in a workspace's status block (tuning aid)."""
+    buf = (ctypes.c_uint32 * 5)()
+    _check(lib().fp8idx_read_device_stats(_ptr(workspace), buf, 5, _stream(stream)))
+    return dict(status=buf[0], compactions=buf[1], general_selects=buf[2], candidates=buf[3],
+                max_boundary=buf[4])
 
 
 # ---------------------------------------------------------------------------- calls

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -101,18 +102,31 @@ struct Plan {
   int num_units = 0;
   int grid = 0;
   int cap = 0;
-  size_t off_cand = 0, off_part = 0, off_cnt = 0, total = 0;
+  size_t off_cand = 0, off_scratch = 0, off_part = 0, off_cnt = 0, total = 0;
 };
 
-int candidate_capacity(int topk) { return static_cast<int>(round_up(4 * topk + 256, 128)); }
+// Room for the candidates a row collects over `keys` keys.  With a running
+// threshold at the k-th value seen so far, a key enters with probability
+// about min(1, k / position), so about k * (1 + ln(keys / k)) keys enter in
+// all; half again of that covers the histogram's bin slack.  Overflow is
+// still handled (an exact compaction in the kernel), only slower.
+int candidate_capacity(int topk, int64_t keys) {
+  const double ratio = std::max(1.0, static_cast<double>(keys) / topk);
+  const double expect = topk * (1.0 + std::log(ratio));
+  const int64_t cap = static_cast<int64_t>(1.5 * expect) + 2 * kBlockKeys;
+  return static_cast<int>(round_up(std::max<int64_t>(cap, 2 * topk + 2 * kBlockKeys), kBlockKeys));
+}
 
-void finish_plan(Plan& pl, int64_t groups, int sms, int topk) {
+void finish_plan(Plan& pl, int64_t groups, int sms, int topk, int64_t axis) {
   pl.num_units = static_cast<int>(groups * pl.n_chunks);
   pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(pl.num_units, sms)));
-  pl.cap = candidate_capacity(topk);
+  pl.cap = candidate_capacity(topk, std::min<int64_t>(axis, pl.chunk_keys));
   size_t off = kStatusBytes;
   pl.off_cand = off;
-  off += round_up(static_cast<int64_t>(sms) * pl.R * pl.cap * 8, 256);
+  // two row-state slots per CTA (a unit is selected while the next one streams)
+  off += round_up(static_cast<int64_t>(2) * sms * pl.R * pl.cap * 8, 256);
+  pl.off_scratch = off;  // staging for a rare in-kernel compaction, per epilogue warp
+  off += round_up(static_cast<int64_t>(sms) * 8 * topk * 8, 256);
   if (pl.n_chunks > 1) {
     pl.off_part = off;
     off += round_up(static_cast<int64_t>(pl.num_units) * pl.R * topk * 8, 256);
@@ -137,7 +151,7 @@ Plan plan_prefill(int64_t m, int64_t n, int topk, int sms) {
     pl.chunk_keys = static_cast<int>(ck);
     pl.n_chunks = static_cast<int>(ceil_div(axis, ck));
   }
-  finish_plan(pl, groups, sms, topk);
+  finish_plan(pl, groups, sms, topk, axis);
   return pl;
 }
 
@@ -155,7 +169,7 @@ Plan plan_paged(int64_t B, int R, int max_blocks, int topk, int sms) {
     pl.chunk_keys = static_cast<int>(ck);
     pl.n_chunks = static_cast<int>(ceil_div(axis, ck));
   }
-  finish_plan(pl, B, sms, topk);
+  finish_plan(pl, B, sms, topk, axis);
   return pl;
 }
 
@@ -315,6 +329,7 @@ int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, c
   p.status = reinterpret_cast<int*>(wsb);
   p.cand = reinterpret_cast<uint2*>(wsb + pl.off_cand);
   p.cand_cap = pl.cap;
+  p.scratch = reinterpret_cast<uint2*>(wsb + pl.off_scratch);
   if (pl.n_chunks > 1) {
     p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
     p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
@@ -399,6 +414,7 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
   p.status = reinterpret_cast<int*>(wsb);
   p.cand = reinterpret_cast<uint2*>(wsb + pl.off_cand);
   p.cand_cap = pl.cap;
+  p.scratch = reinterpret_cast<uint2*>(wsb + pl.off_scratch);
   if (pl.n_chunks > 1) {
     p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
     p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
@@ -411,6 +427,15 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
     e = launch_merge(mp, st);
     if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }
+  return ok();
+}
+
+int fp8idx_read_device_stats(const void* ws, uint32_t* out, int count, void* stream) {
+  if (!ws || !out || count < 1 || count > kStatusBytes / 4) return fail(FP8IDX_EINVAL, "bad arguments");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(out, ws, sizeof(uint32_t) * count, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "stats read");
   return ok();
 }
 

@@ -19,11 +19,19 @@
 //               weights and the key scale, then either writes the logit
 //               (mqa_logits) or filters it against the row's running
 //               threshold into a per-row candidate buffer (fused top-k).
+//               A 512-bin histogram of each row's candidates (window opened
+//               on the row's first candidates) raises the threshold to the
+//               lower edge of the bin that holds the k-th candidate.
+//   warps 10..11 select group (fused top-k): takes a finished unit's row
+//               state (double buffered, so it overlaps the next unit) and
+//               selects each row's exact top-k: keys above the boundary bin
+//               go straight out, the boundary bin is resolved in shared memory.
 // A unit is R query rows (a row block, or one request's rows in the paged
 // form) times one chunk of keys.  With one chunk per unit the fused kernel
 // writes the final top-k; with several, each unit writes its exact partial
 // top-k and the merge kernel selects from the union.
 #include <cfloat>
+#include <climits>
 #include <cstdint>
 
 #include "kernels.cuh"
@@ -36,7 +44,7 @@ template <int R, bool PAGED>
 struct Cfg {
   static constexpr int N = R * kHeads;         // MMA N: (row, head) columns
   static constexpr int RW = R / 2;             // rows per epilogue warpgroup
-  static constexpr int STAGES = PAGED ? 8 : 5; // key-tile ring depth
+  static constexpr int STAGES = PAGED ? (R == 8 ? 5 : 7) : 5;  // key-tile ring depth
   static constexpr int Q_BYTES = N * kDim;
   static constexpr int TILE_BYTES = kBlockKeys * kDim;
   static constexpr int TMEM_COLS = 2 * N;
@@ -45,10 +53,40 @@ struct Cfg {
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns must be a power of two");
 };
 
-constexpr int kSelWords = 264;  // per epilogue warp: hist[256], counter, pad
+constexpr int kNB = 512;         // histogram bins per row
+constexpr int kSelWords = 264;   // per epilogue warp: hist[256], counter, pad
+constexpr int kSelWG = 10;       // first warp of the select group
+constexpr int kSelWarps = 2;     // warps in the select group
+constexpr int kSelBar = 3;       // its named barrier
+constexpr int kUpCap = kMaxTopK; // per select warp: keys above the boundary bin (fewer than topk in all)
+constexpr int kAtCap = 1024;     // per select warp: keys inside the boundary bin
+
+// Per (slot, row) streaming state of the fused top-k.  A row's candidate
+// buffer holds four equal segments, one per TMEM lane quadrant (key block of
+// 32 inside each tile), so each epilogue warp appends with a private counter.
+struct RowState {
+  int wcnt[4];     // candidates in each segment
+  uint32_t theta;  // keep a key only if order_key >= theta
+  float theta_f;   // the float whose order key is theta (-inf when theta admits all)
+  uint32_t base;   // histogram window: bin = min((key - base) >> shift, kNB - 1)
+  int shift;
+  int mode;        // 0: window not set yet, 1: histogram live
+  uint32_t tmin;   // min / max key collected while the window is not set
+  uint32_t tmax;
+  int lo, hi;      // the row's key range inside this unit's chunk
+  int pad[2];
+};
+
+__device__ __forceinline__ float theta_float(uint32_t key) {
+  return key <= 0x007FFFFFu ? -INFINITY : key_to_float(key);
+}
+
+struct SlotMeta {
+  int unit, row0, nrows, pad;
+};
 
 struct SmemLayout {
-  int q, stage, bar, misc, w, rows, sel, total;
+  int q, stage, bar, misc, w, rows, meta, hist, esel, ssel, up, at, total;
 };
 
 template <int R, bool PAGED>
@@ -58,11 +96,16 @@ __host__ __device__ constexpr SmemLayout smem_layout() {
   L.q = 0;
   L.stage = C::Q_BYTES;
   L.bar = L.stage + C::STAGES * C::TILE_BYTES;
-  L.misc = L.bar + 8 * (2 * C::STAGES + 8);
+  L.misc = L.bar + 8 * (2 * C::STAGES + 12);
   L.w = L.misc + 64;
   L.rows = L.w + R * kHeads * 4;
-  L.sel = L.rows + 2 * R * 4;
-  L.total = L.sel + 8 * kSelWords * 4;
+  L.meta = L.rows + 2 * R * static_cast<int>(sizeof(RowState));
+  L.hist = L.meta + 2 * static_cast<int>(sizeof(SlotMeta));
+  L.esel = L.hist + 2 * R * kNB * 4;
+  L.ssel = L.esel + 8 * kSelWords * 4;
+  L.up = L.ssel + 320 * 4;
+  L.at = L.up + kSelWarps * kUpCap * 8;
+  L.total = L.at + kSelWarps * kAtCap * 8;
   return L;
 }
 
@@ -72,11 +115,12 @@ struct Unit {
   int row0;      // first query row
   int nrows;     // rows present (<= R)
   int req;       // paged: request
-  int64_t cbeg;  // chunk [cbeg, cend) of the key axis
-  int64_t cend;
-  int64_t jbeg;  // first key of the first tile
+  int cbeg;      // chunk [cbeg, cend) of the key axis
+  int cend;
+  int jbeg;      // first key of the first tile
   int ntiles;
-  int64_t len;   // paged: context length (clamped)
+  int len;       // paged: context length (clamped)
+  bool len_clamped;
 };
 
 template <int R, bool PAGED>
@@ -87,14 +131,15 @@ __device__ __forceinline__ Unit get_unit(const IndexerParams& p, int u) {
   U.row0 = grp * R;
   U.nrows = min(R, p.m - U.row0);
   U.req = grp;
-  int64_t lo, hi, axis;
+  U.len_clamped = false;
+  int lo, hi, axis;
   if (!PAGED) {
-    axis = p.n;
-    lo = INT64_MAX;
-    hi = INT64_MIN;
+    axis = static_cast<int>(p.n);
+    lo = INT_MAX;
+    hi = INT_MIN;
     for (int r = 0; r < U.nrows; ++r) {
-      int64_t a = max(static_cast<int64_t>(__ldg(p.ks + U.row0 + r)), static_cast<int64_t>(0));
-      int64_t b = min(static_cast<int64_t>(__ldg(p.ke + U.row0 + r)), p.n);
+      const int a = max(__ldg(p.ks + U.row0 + r), 0);
+      const int b = min(__ldg(p.ke + U.row0 + r), axis);
       if (b > a) {
         lo = min(lo, a);
         hi = max(hi, b);
@@ -102,18 +147,18 @@ __device__ __forceinline__ Unit get_unit(const IndexerParams& p, int u) {
     }
     U.len = 0;
   } else {
-    axis = static_cast<int64_t>(p.max_blocks) * kPageSize;
-    int64_t L = __ldg(p.seq_lens + grp);
-    L = max(min(L, axis), static_cast<int64_t>(0));
-    U.len = L;
+    axis = p.max_blocks * kPageSize;
+    const int L = __ldg(p.seq_lens + grp);
+    U.len_clamped = L > axis;
+    U.len = max(min(L, axis), 0);
     lo = 0;
-    hi = L;
+    hi = U.len;
   }
-  U.cbeg = static_cast<int64_t>(c) * p.chunk_keys;
+  U.cbeg = c * p.chunk_keys;
   U.cend = min(U.cbeg + p.chunk_keys, axis);
-  const int64_t jb = max(U.cbeg, lo), je = min(U.cend, hi);
+  const int jb = max(U.cbeg, lo), je = min(U.cend, hi);
   U.jbeg = jb;
-  U.ntiles = je > jb ? static_cast<int>((je - jb + kBlockKeys - 1) / kBlockKeys) : 0;
+  U.ntiles = je > jb ? (je - jb + kBlockKeys - 1) / kBlockKeys : 0;
   return U;
 }
 
@@ -123,16 +168,13 @@ __device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile i
                                       int* status, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  uint32_t it = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++it & 31) == 0) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > limit_ns) {
-        *abort_flag = 1;
-        atomicOr(status, kStatusWaitTimeout);
-        return false;
-      }
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(status, kStatusWaitTimeout);
+      return false;
     }
   }
 }
@@ -151,30 +193,238 @@ __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
   return r != 0;
 }
 
-// sum_h w[h] * max(x[h], 0) over the 32 heads of one (key, row).
+// Uniform count of the threads of a named barrier whose predicate is set.
+__device__ __forceinline__ uint32_t bar_red_popc(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.popc.u32 %0, %2, %3, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r;
+}
+
+// sum_h w[h] * max(x[h], 0) over the 32 heads of one (key, row), with packed
+// two-lane fp32 FMAs (each lane rounded once, like fmaf).
 __device__ __forceinline__ float relu_dot32(const uint32_t (&x)[32], const float* wsm) {
   const float4* w4 = reinterpret_cast<const float4*>(wsm);
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  uint64_t a0 = 0, a1 = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 wv = w4[i];
-    a0 = fmaf(wv.x, fmaxf(__uint_as_float(x[4 * i + 0]), 0.f), a0);
-    a1 = fmaf(wv.y, fmaxf(__uint_as_float(x[4 * i + 1]), 0.f), a1);
-    a2 = fmaf(wv.z, fmaxf(__uint_as_float(x[4 * i + 2]), 0.f), a2);
-    a3 = fmaf(wv.w, fmaxf(__uint_as_float(x[4 * i + 3]), 0.f), a3);
+    const uint64_t r01 = pack_f32x2(fmaxf(__uint_as_float(x[4 * i + 0]), 0.f),
+                                    fmaxf(__uint_as_float(x[4 * i + 1]), 0.f));
+    const uint64_t r23 = pack_f32x2(fmaxf(__uint_as_float(x[4 * i + 2]), 0.f),
+                                    fmaxf(__uint_as_float(x[4 * i + 3]), 0.f));
+    a0 = fma_f32x2(pack_f32x2(wv.x, wv.y), r01, a0);
+    a1 = fma_f32x2(pack_f32x2(wv.z, wv.w), r23, a1);
   }
-  return (a0 + a1) + (a2 + a3);
+  float s0, s1, s2, s3;
+  unpack_f32x2(a0, s0, s1);
+  unpack_f32x2(a1, s2, s3);
+  return (s0 + s1) + (s2 + s3);
 }
 
-// A row's candidate buffer as a select source.
-struct BufSrc {
+// Histogram slot of bin b: lane (b >> 4) owns bins [16 lane, 16 lane + 16),
+// stored transposed so that a warp reading one bin per lane hits 32 banks.
+__device__ __forceinline__ int hist_index(int b) { return (b & 15) * 32 + (b >> 4); }
+
+__device__ __forceinline__ int hist_bin(uint32_t key, uint32_t base, int shift) {
+  return static_cast<int>(min((key - base) >> shift, static_cast<uint32_t>(kNB - 1)));
+}
+
+// Find the boundary bin: the highest bin b such that at least k counted
+// candidates lie in bins >= b.  Every lane returns the same result.
+struct Boundary {
+  bool found;
+  int bin;
+  uint32_t above;  // candidates in bins > bin
+  uint32_t inbin;
+};
+
+__device__ __forceinline__ Boundary find_boundary(const uint32_t* h, uint32_t k, int lane) {
+  uint32_t c[16];
+  uint32_t tot = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    c[i] = h[i * 32 + lane];
+    tot += c[i];
+  }
+  uint32_t suf = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t t = __shfl_down_sync(0xFFFFFFFFu, suf, off);
+    if (lane + off < 32) suf += t;
+  }
+  Boundary B{false, 0, 0, 0};
+  const uint32_t ball = __ballot_sync(0xFFFFFFFFu, suf >= k);
+  if (ball == 0) return B;
+  const int ls = 31 - __clz(static_cast<int>(ball));
+  int bin = 0;
+  uint32_t above = 0, inbin = 0;
+  if (lane == ls) {
+    uint32_t run = suf - tot;
+#pragma unroll
+    for (int i = 15; i >= 0; --i) {
+      if (run + c[i] >= k) {
+        bin = ls * 16 + i;
+        inbin = c[i];
+        break;
+      }
+      run += c[i];
+    }
+    above = run;
+  }
+  B.found = true;
+  B.bin = __shfl_sync(0xFFFFFFFFu, bin, ls);
+  B.above = __shfl_sync(0xFFFFFFFFu, above, ls);
+  B.inbin = __shfl_sync(0xFFFFFFFFu, inbin, ls);
+  return B;
+}
+
+// A row's four candidate segments as a select source (positions [0, 4 * wcap)).
+struct SegSrc {
   const uint2* buf;
+  int wcap;
+  int c0, c1, c2, c3;
   __device__ __forceinline__ bool get(int e, uint64_t& K) const {
+    const int s = e / wcap;
+    const int i = e - s * wcap;
+    const int c = s == 0 ? c0 : s == 1 ? c1 : s == 2 ? c2 : c3;
+    if (i >= c) return false;
     const uint2 v = buf[e];
     K = compose_key(v.x, v.y);
     return true;
   }
 };
+
+// Two shared-memory lists back to back as a select source.
+struct TwoListSrc {
+  const uint2* a;
+  int na;
+  const uint2* b;
+  int nb;
+  __device__ __forceinline__ bool get(int e, uint64_t& K) const {
+    uint2 v;
+    if (e < na)
+      v = a[e];
+    else if (e - na < nb)
+      v = b[e - na];
+    else
+      return false;
+    K = compose_key(v.x, v.y);
+    return true;
+  }
+};
+
+// Exact top-k of one finished row by the select group (two warps; warp w
+// reads segments 2w and 2w+1).  emit(pos, key, index) receives positions
+// [0, returned count).  Keys above the histogram's boundary bin are in; the
+// boundary bin is resolved exactly in shared memory; anything unusual falls
+// back to a radix select over the whole buffer.
+template <class Emit>
+__device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& st, const uint32_t* h,
+                                int k, const Group<kSelWarps>& g, uint2* up_all, uint2* at_all,
+                                uint32_t* xchg, int* stats, Emit emit) {
+  const int w = g.warp(), lane = g.lane();
+  const int c[4] = {st.wcnt[0], st.wcnt[1], st.wcnt[2], st.wcnt[3]};
+  const int cnt = c[0] + c[1] + c[2] + c[3];
+  if (cnt <= k) {
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int s = 2 * w + s2;
+      const int pref = (s > 0 ? c[0] : 0) + (s > 1 ? c[1] : 0) + (s > 2 ? c[2] : 0);
+      const uint2* seg = rowbuf + s * wcap;
+      for (int i0 = 0; i0 < c[s]; i0 += 8 * 32) {
+        uint2 v[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int i = i0 + t * 32 + lane;
+          if (i < c[s]) v[t] = seg[i];
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int i = i0 + t * 32 + lane;
+          if (i < c[s]) emit(pref + i, v[t].x, v[t].y);
+        }
+      }
+    }
+    return cnt;
+  }
+  if (st.mode == 1) {
+    const Boundary B = find_boundary(h, static_cast<uint32_t>(k), lane);
+    if (B.found) {
+      if (g.tid == 0) atomicMax(reinterpret_cast<unsigned*>(stats + kStatMaxBoundary), B.inbin);
+      uint2* up_w = up_all + w * kUpCap;
+      uint2* at_w = at_all + w * kAtCap;
+      uint32_t nu = 0, na = 0;  // warp-uniform counters
+      const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const int s = 2 * w + s2;
+        const uint2* seg = rowbuf + s * wcap;
+        for (int i0 = 0; i0 < c[s]; i0 += 8 * 32) {
+          uint2 v[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int i = i0 + t * 32 + lane;
+            v[t] = i < c[s] ? seg[i] : make_uint2(0u, 0u);
+          }
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int i = i0 + t * 32 + lane;
+            int bin = -1;
+            if (i < c[s] && v[t].x >= st.base) bin = hist_bin(v[t].x, st.base, st.shift);
+            const bool up = bin > B.bin, at = bin == B.bin;
+            const uint32_t mu = __ballot_sync(0xFFFFFFFFu, up);
+            const uint32_t ma = __ballot_sync(0xFFFFFFFFu, at);
+            if (up) {
+              const uint32_t q = nu + __popc(mu & lt);
+              if (q < static_cast<uint32_t>(kUpCap)) up_w[q] = v[t];
+            }
+            if (at) {
+              const uint32_t q = na + __popc(ma & lt);
+              if (q < static_cast<uint32_t>(kAtCap)) at_w[q] = v[t];
+            }
+            nu += __popc(mu);
+            na += __popc(ma);
+          }
+        }
+      }
+      if (lane == 0) {
+        xchg[2 * w] = nu;
+        xchg[2 * w + 1] = na;
+      }
+      g.sync();
+      const uint32_t nu0 = xchg[0], na0 = xchg[1], nu1 = xchg[2], na1 = xchg[3];
+      const bool consistent = nu0 + nu1 == B.above && na0 + na1 == B.inbin &&
+                              nu0 <= static_cast<uint32_t>(kUpCap) && nu1 <= static_cast<uint32_t>(kUpCap) &&
+                              na0 <= static_cast<uint32_t>(kAtCap) && na1 <= static_cast<uint32_t>(kAtCap);
+      if (consistent) {
+        const uint32_t off = w == 0 ? 0u : nu0;
+        const uint32_t mine = w == 0 ? nu0 : nu1;
+        for (uint32_t i = lane; i < mine; i += 32) emit(static_cast<int>(off + i), up_w[i].x, up_w[i].y);
+        const int need = k - static_cast<int>(B.above);
+        const TwoListSrc src{at_all, static_cast<int>(na0), at_all + kAtCap, static_cast<int>(na1)};
+        const int tot = static_cast<int>(na0 + na1);
+        const SelectResult sel = group_select<kSelWarps>(src, tot, need, g);
+        const int n2 = group_emit<kSelWarps>(src, tot, sel, g, [&](int pos, uint64_t K) {
+          emit(static_cast<int>(B.above) + pos, composite_value(K), composite_index(K));
+        });
+        return static_cast<int>(B.above) + n2;
+      }
+    }
+  }
+  // general path: radix select over the whole buffer
+  if (g.tid == 0) atomicAdd(stats + kStatGeneralSelects, 1);
+  const SegSrc src{rowbuf, wcap, c[0], c[1], c[2], c[3]};
+  const SelectResult sel = group_select<kSelWarps>(src, 4 * wcap, k, g);
+  return group_emit<kSelWarps>(src, 4 * wcap, sel, g, [&](int pos, uint64_t K) {
+    emit(pos, composite_value(K), composite_index(K));
+  });
+}
 
 // ------------------------------------------------------------------ kernel
 
@@ -199,12 +449,18 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
   uint64_t* qfull = bars + 2 * S + 4;
   uint64_t* qempty = bars + 2 * S + 5;
   uint64_t* drain = bars + 2 * S + 6;
+  uint64_t* slot_full = bars + 2 * S + 7;
+  uint64_t* slot_empty = bars + 2 * S + 9;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SL.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL.misc + 4);
   float* w_smem = reinterpret_cast<float*>(smem + SL.w);
-  int* cnt_smem = reinterpret_cast<int*>(smem + SL.rows);
-  uint32_t* theta_smem = reinterpret_cast<uint32_t*>(smem + SL.rows + R * 4);
-  uint32_t* sel_smem = reinterpret_cast<uint32_t*>(smem + SL.sel);
+  RowState* rstate = reinterpret_cast<RowState*>(smem + SL.rows);
+  SlotMeta* smeta = reinterpret_cast<SlotMeta*>(smem + SL.meta);
+  uint32_t* hist_smem = reinterpret_cast<uint32_t*>(smem + SL.hist);
+  uint32_t* esel_smem = reinterpret_cast<uint32_t*>(smem + SL.esel);
+  uint32_t* ssel_smem = reinterpret_cast<uint32_t*>(smem + SL.ssel);
+  uint2* up_smem = reinterpret_cast<uint2*>(smem + SL.up);
+  uint2* at_smem = reinterpret_cast<uint2*>(smem + SL.at);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -217,6 +473,8 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 8);
+      mbar_init(&slot_full[a], 8);
+      mbar_init(&slot_empty[a], kSelWarps);
     }
     mbar_init(qfull, 1);
     mbar_init(qempty, 1);
@@ -257,21 +515,22 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         qphase ^= 1;
         mbar_arrive_expect_tx(qfull, C::Q_BYTES);
         tma_load_2d(q_smem, &p.tmap_q, qfull, 0, U.row0 * kHeads);
+        const int32_t* bt = PAGED ? p.block_table + static_cast<int64_t>(U.req) * p.max_blocks : nullptr;
         for (int t = 0; t < U.ntiles; ++t) {
           if (!wait_bar(&empty[stage], phase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
-          const int64_t j0 = U.jbeg + static_cast<int64_t>(t) * kBlockKeys;
+          const int j0 = U.jbeg + t * kBlockKeys;
           uint8_t* dst = stage_smem + stage * C::TILE_BYTES;
           if (!PAGED) {
             mbar_arrive_expect_tx(&full[stage], C::TILE_BYTES);
-            tma_load_2d(dst, &p.tmap_k, &full[stage], 0, static_cast<int32_t>(j0));
+            tma_load_2d(dst, &p.tmap_k, &full[stage], 0, j0);
           } else {
-            const int64_t lp = j0 / kPageSize;
-            const int32_t* bt = p.block_table + static_cast<int64_t>(U.req) * p.max_blocks;
-            int32_t pg0 = __ldg(bt + lp);
-            int32_t pg1 = (j0 + kPageSize < U.len) ? __ldg(bt + lp + 1) : -1;
-            bool v0 = pg0 >= 0 && pg0 < p.num_pages;
-            bool v1 = pg1 >= 0 && pg1 < p.num_pages;
-            if (!v0 || (j0 + kPageSize < U.len && !v1)) atomicOr(p.status, kStatusBadPage);
+            const int lp = j0 / kPageSize;
+            const bool has1 = j0 + kPageSize < U.len;
+            const int32_t pg0 = __ldg(bt + lp);
+            const int32_t pg1 = has1 ? __ldg(bt + lp + 1) : -1;
+            const bool v0 = pg0 >= 0 && pg0 < p.num_pages;
+            const bool v1 = has1 && pg1 >= 0 && pg1 < p.num_pages;
+            if (!v0 || (has1 && !v1)) atomicOr(p.status, kStatusBadPage);
             mbar_arrive_expect_tx(&full[stage], (v0 ? 8192u : 0u) + (v1 ? 8192u : 0u));
             if (v0) tma_load_2d(dst, &p.tmap_k, &full[stage], 0, pg0 * kPageSize);
             if (v1) tma_load_2d(dst + 8192, &p.tmap_k, &full[stage], 0, pg1 * kPageSize);
@@ -338,78 +597,106 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         }
       }
     }
-  } else {
+  } else if (warp < kSelWG) {
     // ---------------------------------------------------------------- epilogue
     const int ew = warp - 2;  // 0..7
     const int g = ew >> 2;    // warpgroup
-    const int qd = warp & 3;  // TMEM lane quadrant == key block of 32
+    const int qd = warp & 3;  // TMEM lane quadrant == key block of 32 == buffer segment
     const int tid_wg = qd * 32 + lane;
     const int bar_id = 1 + g;
     float* ws_g = w_smem + g * RW * kHeads;
-    int* cnt_g = cnt_smem + g * RW;
-    uint32_t* th_g = theta_smem + g * RW;
-    Group<1> grp{sel_smem + ew * kSelWords, nullptr, sel_smem + ew * kSelWords + 256, 0, lane};
+    Group<1> grp{esel_smem + ew * kSelWords, nullptr, esel_smem + ew * kSelWords + 256, 0, lane};
     const int k = p.topk;
     const int cap = p.cand_cap;
-    uint2* cand_g = p.cand ? p.cand + (static_cast<size_t>(blockIdx.x) * R + g * RW) * cap : nullptr;
+    const int wcap = cap >> 2;  // segment capacity
     const uint32_t lane_addr = tbase + (static_cast<uint32_t>(qd * 32) << 16);
+    const uint32_t lt = (1u << lane) - 1u;
     uint32_t T = 0;
     bool aborted = false;
 
-    for (int i = blockIdx.x; i < p.num_units; i += gridDim.x) {
+    for (int i = blockIdx.x, it = 0; i < p.num_units; i += gridDim.x, ++it) {
       const int u = p.num_units - 1 - i;
       const Unit U = get_unit<R, PAGED>(p, u);
-      // ---- per-row setup for this warpgroup's rows
-      int64_t lo_r[RW], hi_r[RW];
-      bool rv[RW];
-#pragma unroll
-      for (int r = 0; r < RW; ++r) {
-        const int rl = g * RW + r;
-        rv[r] = rl < U.nrows;
-        lo_r[r] = 0;
-        hi_r[r] = 0;
-        if (rv[r]) {
+      const int slot = it & 1;
+      RowState* rs = rstate + slot * R + g * RW;
+      uint32_t* hs = hist_smem + (slot * R + g * RW) * kNB;
+      uint2* cand_s = MODE == kModeTopK
+                          ? p.cand + (static_cast<size_t>(blockIdx.x * 2 + slot) * R + g * RW) * cap
+                          : nullptr;
+      if (MODE == kModeTopK) {
+        if (!wait_bar(&slot_empty[slot], ((it >> 1) & 1) ^ 1, abort_flag, p.status, limit)) aborted = true;
+      }
+      // ---- per-row setup for this warpgroup's rows: the key range [lo, hi)
+      // (kept in shared memory; the tile loop reads it back as a broadcast)
+      if (tid_wg < RW) {
+        const int rl = g * RW + tid_wg;
+        int lo = 0, hi = 0;
+        if (rl < U.nrows) {
           const int row = U.row0 + rl;
           if (!PAGED) {
-            int64_t a = max(static_cast<int64_t>(__ldg(p.ks + row)), static_cast<int64_t>(0));
-            int64_t b = min(static_cast<int64_t>(__ldg(p.ke + row)), p.n);
-            lo_r[r] = a;
-            hi_r[r] = max(a, b);
+            lo = max(__ldg(p.ks + row), 0);
+            hi = max(lo, min(__ldg(p.ke + row), static_cast<int>(p.n)));
           } else {
-            int64_t e = U.len - R + rl + 1;
-            hi_r[r] = max(min(e, U.len), static_cast<int64_t>(0));
+            const int e = U.len - R + rl + 1;
+            hi = max(min(e, U.len), 0);
           }
           // a unit only owns the keys of its chunk (its last tile may overhang)
-          lo_r[r] = max(lo_r[r], U.cbeg);
-          hi_r[r] = min(hi_r[r], U.cend);
+          lo = max(lo, U.cbeg);
+          hi = max(lo, min(hi, U.cend));
         }
+        rs[tid_wg].lo = lo;
+        rs[tid_wg].hi = hi;
       }
       if (tid_wg < RW * kHeads) {
         const int rl = g * RW + tid_wg / kHeads;
         ws_g[tid_wg] = rl < U.nrows ? __ldg(p.w + static_cast<int64_t>(U.row0 + rl) * kHeads + tid_wg % kHeads) : 0.f;
       }
-      if (tid_wg < RW) {
-        cnt_g[tid_wg] = 0;
-        th_g[tid_wg] = 0;
+      if (MODE == kModeTopK) {
+        if (tid_wg < RW) {
+          RowState& st = rs[tid_wg];
+          st.wcnt[0] = st.wcnt[1] = st.wcnt[2] = st.wcnt[3] = 0;
+          st.theta = 0;
+          st.theta_f = -INFINITY;
+          st.base = 0;
+          st.shift = 0;
+          st.mode = 0;
+          st.tmin = 0xFFFFFFFFu;
+          st.tmax = 0;
+        }
+        for (int x = tid_wg; x < RW * kNB; x += 128) hs[x] = 0;
+        if (g == 0 && tid_wg == 0) {
+          smeta[slot].unit = u;
+          smeta[slot].row0 = U.row0;
+          smeta[slot].nrows = U.nrows;
+          if (PAGED && U.len_clamped) atomicOr(p.status, kStatusSeqLenTooLong);
+        }
       }
-      named_bar_sync(bar_id, 128);
+      if (bar_red_or(bar_id, 128, aborted || *abort_flag)) {
+        aborted = true;
+        break;
+      }
 
       if (MODE == kModeLogits) {
         // keys of this chunk that no tile covers are -inf
-        const int64_t tb = U.ntiles ? U.jbeg : U.cend;
-        const int64_t te = U.ntiles ? U.jbeg + static_cast<int64_t>(U.ntiles) * kBlockKeys : U.cend;
+        const int tb = U.ntiles ? U.jbeg : U.cend;
+        const int te = U.ntiles ? U.jbeg + U.ntiles * kBlockKeys : U.cend;
 #pragma unroll
         for (int r = 0; r < RW; ++r) {
-          if (!rv[r]) continue;
+          if (g * RW + r >= U.nrows) continue;
           float* lrow = p.logits + static_cast<int64_t>(U.row0 + g * RW + r) * p.ld_logits;
-          for (int64_t j = U.cbeg + tid_wg; j < U.cend; j += 128)
+          for (int j = U.cbeg + tid_wg; j < U.cend; j += 128)
             if (j < tb || j >= te) __stcs(lrow + j, -INFINITY);
         }
       }
 
+      // ---- this warp's segment counts (reloaded after maintenance)
+      int wcnt[RW];
+#pragma unroll
+      for (int r = 0; r < RW; ++r) wcnt[r] = 0;
+
       // ---- stream the unit's key tiles
-      const int64_t key0 = U.jbeg + qd * 32 + lane;
-      auto scale_of = [&](int64_t j) -> float {
+      const int key0 = U.jbeg + qd * 32 + lane;
+      auto scale_of = [&](int j) -> float {
         if (!PAGED) return j < p.n ? __ldg(p.s + j) : 0.f;
         if (j >= U.len) return 0.f;
         const int32_t pg = __ldg(p.block_table + static_cast<int64_t>(U.req) * p.max_blocks + j / kPageSize);
@@ -417,8 +704,9 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         return __ldg(p.s + static_cast<int64_t>(pg) * kPageSize + (j % kPageSize));
       };
       float s_next = U.ntiles ? scale_of(key0) : 0.f;
+      bool maint = false;  // this warp saw a row that needs maintenance at the next vote
       for (int t = 0; t < U.ntiles; ++t, ++T) {
-        const int64_t j = key0 + static_cast<int64_t>(t) * kBlockKeys;
+        const int j = key0 + t * kBlockKeys;
         const float sj = s_next;
         if (t + 1 < U.ntiles) s_next = scale_of(j + kBlockKeys);
         const uint32_t a = T & 1, aph = (T >> 1) & 1;
@@ -426,110 +714,224 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         tc_fence_after();
         float L[RW];
 #pragma unroll
-        for (int r = 0; r < RW; ++r) {
-          uint32_t x[32];
-          tmem_ld32(lane_addr + a * N + (g * RW + r) * kHeads, x);
+        for (int r = 0; r < RW; r += 2) {  // two rows (64 columns) per TMEM read
+          uint32_t x0[32], x1[32];
+          tmem_ld32(lane_addr + a * N + (g * RW + r) * kHeads, x0);
+          tmem_ld32(lane_addr + a * N + (g * RW + r + 1) * kHeads, x1);
           tmem_ld_wait();
-          L[r] = relu_dot32(x, ws_g + r * kHeads) * sj;
+          if (r + 2 == RW) {  // the accumulator is in registers now
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[a]);
+          }
+          L[r] = relu_dot32(x0, ws_g + r * kHeads) * sj;
+          L[r + 1] = relu_dot32(x1, ws_g + (r + 1) * kHeads) * sj;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[a]);
 
         if (MODE == kModeLogits) {
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
-            if (!rv[r] || j >= U.cend) continue;
+            if (g * RW + r >= U.nrows || j >= U.cend) continue;
             float* lrow = p.logits + static_cast<int64_t>(U.row0 + g * RW + r) * p.ld_logits;
-            __stcs(lrow + j, (j >= lo_r[r] && j < hi_r[r]) ? L[r] : -INFINITY);
+            __stcs(lrow + j, (j >= rs[r].lo && j < rs[r].hi) ? L[r] : -INFINITY);
           }
           if (bar_red_or(bar_id, 128, aborted || *abort_flag)) {
             aborted = true;
             break;
           }
         } else {
+          // ---- filter against the running threshold; append to this warp's segment
+          float thf[RW];
+#pragma unroll
+          for (int r = 0; r < RW; ++r) thf[r] = rs[r].theta_f;
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
-            const uint32_t key = order_key(L[r]);
-            const bool pass = rv[r] && j >= lo_r[r] && j < hi_r[r] && key >= th_g[r];
-            const uint32_t msk = __ballot_sync(0xFFFFFFFFu, pass);
+            const bool ps = j >= rs[r].lo && j < rs[r].hi && L[r] >= thf[r];
+            const uint32_t msk = __ballot_sync(0xFFFFFFFFu, ps);
             if (msk) {
-              const int leader = __ffs(static_cast<int>(msk)) - 1;
-              int base = 0;
-              if (lane == leader) base = atomicAdd(&cnt_g[r], __popc(msk));
-              base = __shfl_sync(0xFFFFFFFFu, base, leader);
-              if (pass)
-                cand_g[static_cast<size_t>(r) * cap + base + __popc(msk & ((1u << lane) - 1u))] =
-                    make_uint2(key, static_cast<uint32_t>(j));
+              const uint32_t key = order_key(L[r]);
+              if (ps) {
+                const int pos = wcnt[r] + __popc(msk & lt);
+                if (pos < wcap)
+                  cand_s[static_cast<size_t>(r) * cap + qd * wcap + pos] = make_uint2(key, static_cast<uint32_t>(j));
+                else
+                  atomicOr(p.status, kStatusCandOverflow);
+              }
+              wcnt[r] += __popc(msk);
+              const RowState& st = rs[r];
+              if (st.mode == 1) {
+                const uint32_t base = st.base;
+                if (ps && key >= base)
+                  atomicAdd(&hs[r * kNB + hist_index(hist_bin(key, base, st.shift))], 1u);
+              } else {
+                const uint32_t wmin = __reduce_min_sync(0xFFFFFFFFu, ps ? key : 0xFFFFFFFFu);
+                const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, ps ? key : 0u);
+                if (lane == 0) {
+                  atomicMin(&rs[r].tmin, wmin);
+                  atomicMax(&rs[r].tmax, wmax);
+                }
+                maint = true;  // the row opens its histogram window at the next vote
+              }
+              if (wcnt[r] > wcap - 64) maint = true;
             }
           }
-          if (bar_red_or(bar_id, 128, aborted || *abort_flag)) {
-            aborted = true;
-            break;
-          }
-          // Keep room for one more tile per row: compact rows that are near full
-          // to their exact top-k; later keys only enter above the k-th value.
-          bool need = false;
+          // Every other tile (and the last), one barrier carries two votes:
+          // abort (weight 1: lane 0 of each warp) and maintenance (weight 5:
+          // lanes 0..4 of each warp).  Between votes a warp adds at most 64
+          // candidates to its segment, which the margin above leaves room for.
+          if ((t & 1) || t + 1 == U.ntiles) {
+            if (lane == 0) {
 #pragma unroll
-          for (int r = 0; r < RW; ++r) need |= cnt_g[r] > cap - kBlockKeys;
-          if (need) {
-            if (qd < RW && cnt_g[qd] > cap - kBlockKeys) {
-              uint2* buf = cand_g + static_cast<size_t>(qd) * cap;
-              const int cnt = cnt_g[qd];
-              const SelectResult sel = group_select<1>(BufSrc{buf}, cnt, k, grp);
-              uint32_t umin = 0xFFFFFFFFu;
-              const int kept = group_emit<1>(BufSrc{buf}, cnt, sel, grp, [&](int pos, uint64_t K) {
-                buf[pos] = make_uint2(composite_value(K), composite_index(K));
-                umin = min(umin, composite_value(K));
-              });
-              umin = __reduce_min_sync(0xFFFFFFFFu, umin);
-              if (lane == 0) {
-                cnt_g[qd] = kept;
-                if (kept >= k) th_g[qd] = max(th_g[qd], umin == 0xFFFFFFFFu ? umin : umin + 1);
+              for (int r = 0; r < RW; ++r) rs[r].wcnt[qd] = min(wcnt[r], wcap);
+            }
+            const bool ab = aborted || *abort_flag;
+            const uint32_t votes = bar_red_popc(bar_id, 128, (lane == 0 && ab) || (lane < 5 && maint));
+            maint = false;
+            if (votes % 5) {
+              aborted = true;
+              break;
+            }
+            if (votes >= 5) {
+              // Quiescent point: every warp of the group is here.  Snapshot, then act.
+              bool opened[RW], compact[RW];
+#pragma unroll
+              for (int r = 0; r < RW; ++r) {
+                const RowState& st = rs[r];
+                opened[r] = st.mode == 0 && st.tmin != 0xFFFFFFFFu;
+                compact[r] = max(max(st.wcnt[0], st.wcnt[1]), max(st.wcnt[2], st.wcnt[3])) > wcap - 64;
+              }
+              named_bar_sync(bar_id, 128);
+              if (qd < RW && (compact[qd] || opened[qd])) {
+                RowState& st = rs[qd];
+                uint2* rowbuf = cand_s + static_cast<size_t>(qd) * cap;
+                uint32_t* h = hs + qd * kNB;
+                if (opened[qd] && lane == 0) {
+                  // window over twice the span of the keys collected so far
+                  const uint64_t span = static_cast<uint64_t>(st.tmax - st.tmin);
+                  const int bits = 64 - __clzll(static_cast<long long>(2 * span + 1));
+                  st.base = st.tmin;
+                  st.shift = bits > 9 ? bits - 9 : 0;
+                  st.mode = 1;
+                }
+                __syncwarp();
+                if (compact[qd]) {
+                  // Rare: a segment is near full.  Keep the row's exact top-k (later keys
+                  // have larger indices, so a key equal to the k-th value never enters
+                  // again), staged through scratch and dealt back over the segments.
+                  const SegSrc src{rowbuf, wcap, st.wcnt[0], st.wcnt[1], st.wcnt[2], st.wcnt[3]};
+                  uint2* scr = p.scratch + (static_cast<size_t>(blockIdx.x) * 8 + ew) * k;
+                  const SelectResult sel = group_select<1>(src, 4 * wcap, k, grp);
+                  uint32_t umin = 0xFFFFFFFFu;
+                  const int kept = group_emit<1>(src, 4 * wcap, sel, grp, [&](int pos, uint64_t K) {
+                    scr[pos] = make_uint2(composite_value(K), composite_index(K));
+                    umin = min(umin, composite_value(K));
+                  });
+                  umin = __reduce_min_sync(0xFFFFFFFFu, umin);
+                  __syncwarp();
+                  for (int pos = lane; pos < kept; pos += 32) rowbuf[(pos & 3) * wcap + (pos >> 2)] = scr[pos];
+                  if (lane == 0) {
+                    for (int s = 0; s < 4; ++s) st.wcnt[s] = (kept - s + 3) / 4;
+                    if (kept >= k) {
+                      st.theta = max(st.theta, umin == 0xFFFFFFFFu ? umin : umin + 1);
+                      st.theta_f = theta_float(st.theta);
+                    }
+                    atomicAdd(p.status + kStatCompactions, 1);
+                  }
+                  for (int x = lane; x < kNB; x += 32) h[x] = 0;
+                  __syncwarp();
+                  for (int e = lane; e < kept; e += 32) {
+                    const uint32_t key = scr[e].x;
+                    if (key >= st.base) atomicAdd(&h[hist_index(hist_bin(key, st.base, st.shift))], 1u);
+                  }
+                } else {
+                  // count the few candidates collected before the window opened
+                  for (int s = 0; s < 4; ++s) {
+                    const uint2* seg = rowbuf + s * wcap;
+                    for (int e = lane; e < st.wcnt[s]; e += 32) {
+                      const uint32_t key = seg[e].x;
+                      if (key >= st.base) atomicAdd(&h[hist_index(hist_bin(key, st.base, st.shift))], 1u);
+                    }
+                  }
+                }
+              }
+              named_bar_sync(bar_id, 128);
+#pragma unroll
+              for (int r = 0; r < RW; ++r) wcnt[r] = rs[r].wcnt[qd];
+            }
+            // ---- raise the threshold from the histogram (one warp per row)
+            if (qd < RW && rs[qd].mode == 1) {
+              RowState& st = rs[qd];
+              const Boundary B = find_boundary(hs + qd * kNB, static_cast<uint32_t>(k), lane);
+              if (B.found && lane == 0) {
+                uint64_t th = static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin) << st.shift);
+                if (th > 0xFFFFFFFFull) th = 0xFFFFFFFFull;
+                if (static_cast<uint32_t>(th) > st.theta) {
+                  st.theta = static_cast<uint32_t>(th);
+                  st.theta_f = theta_float(st.theta);
+                }
               }
             }
-            named_bar_sync(bar_id, 128);
           }
         }
       }
       if (aborted) break;
-
       if (MODE == kModeTopK) {
-        // ---- exact top-k of each row's candidates
-        if (qd < RW) {
-          const int r = qd;
-          const int rl = g * RW + r;
-          const uint2* buf = cand_g + static_cast<size_t>(r) * cap;
-          const int cnt = cnt_g[r];
-          if (p.n_chunks == 1) {
-            if (rl < U.nrows) {
-              const int row = U.row0 + rl;
-              int32_t* orow = p.out_idx + static_cast<int64_t>(row) * k;
-              float* vrow = p.out_vals ? p.out_vals + static_cast<int64_t>(row) * k : nullptr;
-              const SelectResult sel = group_select<1>(BufSrc{buf}, cnt, k, grp);
-              const int nout = group_emit<1>(BufSrc{buf}, cnt, sel, grp, [&](int pos, uint64_t K) {
-                orow[pos] = static_cast<int32_t>(composite_index(K));
-                if (vrow) vrow[pos] = key_to_float(composite_value(K));
-              });
-              for (int pos = nout + lane; pos < k; pos += 32) {
-                orow[pos] = -1;
-                if (vrow) vrow[pos] = -INFINITY;
-              }
-            }
-          } else {
-            uint2* prow = p.part + (static_cast<size_t>(u) * R + rl) * k;
-            int nout = 0;
-            if (rl < U.nrows && cnt > 0) {
-              const SelectResult sel = group_select<1>(BufSrc{buf}, cnt, k, grp);
-              nout = group_emit<1>(BufSrc{buf}, cnt, sel, grp, [&](int pos, uint64_t K) {
-                prow[pos] = make_uint2(composite_value(K), composite_index(K));
-              });
-            }
-            if (lane == 0) p.part_cnt[static_cast<size_t>(u) * R + rl] = nout;
-          }
+        if (lane == 0) {
+#pragma unroll
+          for (int r = 0; r < RW; ++r) rs[r].wcnt[qd] = min(wcnt[r], wcap);
         }
-        named_bar_sync(bar_id, 128);
+        named_bar_sync(bar_id, 128);  // every warp's row-state writes are done
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&slot_full[slot]);
       }
+    }
+  } else if (MODE == kModeTopK) {
+    // ---------------------------------------------------------------- select group
+    const int stid = (warp - kSelWG) * 32 + lane;
+    constexpr int NT = 32 * kSelWarps;
+    Group<kSelWarps> grp{ssel_smem, ssel_smem + 256, ssel_smem + 300, kSelBar, stid};
+    uint32_t* xchg = ssel_smem + 304;
+    const int k = p.topk;
+    const int cap = p.cand_cap;
+    const int wcap = cap >> 2;
+    for (int i = blockIdx.x, it = 0; i < p.num_units; i += gridDim.x, ++it) {
+      const int slot = it & 1;
+      const bool ok = wait_bar(&slot_full[slot], (it >> 1) & 1, abort_flag, p.status, limit);
+      if (bar_red_or(kSelBar, NT, !ok || *abort_flag)) break;
+      const SlotMeta meta = smeta[slot];
+      for (int rl = 0; rl < R; ++rl) {
+        const RowState st = rstate[slot * R + rl];
+        const uint32_t* h = hist_smem + (slot * R + rl) * kNB;
+        const uint2* rowbuf = p.cand + (static_cast<size_t>(blockIdx.x * 2 + slot) * R + rl) * cap;
+        const bool present = rl < meta.nrows;
+        const int cnt = st.wcnt[0] + st.wcnt[1] + st.wcnt[2] + st.wcnt[3];
+        if (present && stid == 0) atomicAdd(p.status + kStatCandidates, cnt);
+        if (p.n_chunks == 1) {
+          if (!present) continue;
+          const int row = meta.row0 + rl;
+          int32_t* orow = p.out_idx + static_cast<int64_t>(row) * k;
+          float* vrow = p.out_vals ? p.out_vals + static_cast<int64_t>(row) * k : nullptr;
+          const int nout = final_select_row(rowbuf, wcap, st, h, k, grp, up_smem, at_smem, xchg, p.status,
+                                            [&](int pos, uint32_t key, uint32_t j) {
+                                              orow[pos] = static_cast<int32_t>(j);
+                                              if (vrow) vrow[pos] = key_to_float(key);
+                                            });
+          for (int pos = nout + stid; pos < k; pos += NT) {
+            orow[pos] = -1;
+            if (vrow) vrow[pos] = -INFINITY;
+          }
+        } else {
+          uint2* prow = p.part + (static_cast<size_t>(meta.unit) * R + rl) * k;
+          int nout = 0;
+          if (present && cnt > 0)
+            nout = final_select_row(rowbuf, wcap, st, h, k, grp, up_smem, at_smem, xchg, p.status,
+                                    [&](int pos, uint32_t key, uint32_t j) { prow[pos] = make_uint2(key, j); });
+          if (stid == 0) p.part_cnt[static_cast<size_t>(meta.unit) * R + rl] = nout;
+        }
+        grp.sync();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&slot_empty[slot]);
     }
   }
 

@@ -12,13 +12,19 @@ constexpr int kDim = 128;          // index head dim (bytes per fp8 row)
 constexpr int kBlockKeys = 128;    // keys per tile = MMA M = TMEM lanes
 constexpr int kPageSize = 64;      // tokens per key page (paged form)
 constexpr int kMaxTopK = 2048;
-constexpr int kThreads = 320;      // 10 warps: TMA, MMA, 8 epilogue
+constexpr int kThreads = 384;      // 12 warps: TMA, MMA, 8 epilogue, 2 select
 constexpr int kStatusBytes = 256;  // device status block at the head of every workspace
 
 // device status bits (workspace word 0)
 constexpr int kStatusWaitTimeout = 1;
 constexpr int kStatusBadPage = 2;
 constexpr int kStatusSeqLenTooLong = 4;
+constexpr int kStatusCandOverflow = 8;
+// device statistics (workspace words 1..) of the fused top-k
+constexpr int kStatCompactions = 1;     // in-stream exact compactions of a full candidate buffer
+constexpr int kStatGeneralSelects = 2;  // final selects that needed the general radix path
+constexpr int kStatCandidates = 3;      // candidates appended, summed over rows
+constexpr int kStatMaxBoundary = 4;     // largest boundary-bin population seen
 
 enum Mode : int { kModeLogits = 0, kModeTopK = 1 };
 
@@ -47,8 +53,9 @@ struct IndexerParams {
   float* out_vals;
   // workspace
   int* status;
-  uint2* cand;      // [gridDim.x][R][cand_cap] (order key, index)
-  int cand_cap;
+  uint2* cand;      // [gridDim.x][2 slots][R][cand_cap] (order key, index); cand_cap % 128 == 0
+  int cand_cap;     // per row; split into 4 equal segments, one per key quadrant
+  uint2* scratch;   // [gridDim.x][8 epilogue warps][topk]: staging of a rare in-kernel compaction
   uint2* part;      // split mode: [num_units][R][topk]
   int* part_cnt;    // split mode: [num_units][R]
   unsigned long long wait_limit_ns;

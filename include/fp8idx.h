@@ -63,7 +63,8 @@ enum {
 enum {
   FP8IDX_STATUS_WAIT_TIMEOUT = 1,   /* a pipeline wait gave up; outputs are invalid      */
   FP8IDX_STATUS_BAD_PAGE = 2,       /* a block-table entry outside [0, num_pages)        */
-  FP8IDX_STATUS_SEQ_TOO_LONG = 4    /* seq_lens[b] > max_blocks * page_size (clamped)    */
+  FP8IDX_STATUS_SEQ_TOO_LONG = 4,   /* seq_lens[b] > max_blocks * page_size (clamped)    */
+  FP8IDX_STATUS_CAND_OVERFLOW = 8   /* internal: a candidate was dropped; outputs invalid */
 };
 
 /*
@@ -140,6 +141,13 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
  * `ws` (ws == NULL: the last fp8idx_mqa_logits call) into *status_out.
  */
 int fp8idx_read_device_status(const void* ws, int* status_out, void* stream);
+/* Copies the first `count` (<= 64) 32-bit words of a workspace's status block:
+ * word 0 the status bits above; for fp8idx_mqa_logits_topk and the paged form,
+ * word 1 the in-kernel compactions of a full candidate buffer, word 2 the rows
+ * whose final selection took the general radix path, word 3 the candidates
+ * collected (summed over rows and key chunks), word 4 the largest
+ * boundary-bin population.  Synchronises `stream`; for tuning and tests. */
+int fp8idx_read_device_stats(const void* ws, uint32_t* out, int count, void* stream);
 /* Message for the last non-OK return on this thread ("" if none). */
 const char* fp8idx_last_error(void);
 /* Number of SMs of the current device (what the workspace sizes assume). */
