@@ -114,7 +114,10 @@ int candidate_capacity(int topk, int64_t keys) {
   const double ratio = std::max(1.0, static_cast<double>(keys) / topk);
   const double expect = topk * (1.0 + std::log(ratio));
   const int64_t cap = static_cast<int64_t>(1.5 * expect) + 2 * kBlockKeys;
-  return static_cast<int>(round_up(std::max<int64_t>(cap, 2 * topk + 2 * kBlockKeys), kBlockKeys));
+  // Each of the row's four segments must hold its share of the k kept by a
+  // compaction plus the 32 keys per tile a warp may add between two votes.
+  const int64_t floor_cap = 2 * static_cast<int64_t>(topk) + 4 * (kVoteTiles + 2) * 32;
+  return static_cast<int>(round_up(std::max<int64_t>(cap, floor_cap), kBlockKeys));
 }
 
 void finish_plan(Plan& pl, int64_t groups, int sms, int topk, int64_t axis) {

@@ -741,45 +741,49 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
           }
         } else {
           // ---- filter against the running threshold; append to this warp's segment
+          int lo[RW], hi[RW], mode[RW], shift[RW];
+          uint32_t base[RW];
           float thf[RW];
 #pragma unroll
-          for (int r = 0; r < RW; ++r) thf[r] = rs[r].theta_f;
+          for (int r = 0; r < RW; ++r) {  // row state, read once per tile
+            const RowState& st = rs[r];
+            lo[r] = st.lo;
+            hi[r] = st.hi;
+            thf[r] = st.theta_f;
+            mode[r] = st.mode;
+            base[r] = st.base;
+            shift[r] = st.shift;
+          }
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
-            const bool ps = j >= rs[r].lo && j < rs[r].hi && L[r] >= thf[r];
+            const bool ps = j >= lo[r] && j < hi[r] && L[r] >= thf[r];
             const uint32_t msk = __ballot_sync(0xFFFFFFFFu, ps);
-            if (msk) {
-              const uint32_t key = order_key(L[r]);
-              if (ps) {
-                const int pos = wcnt[r] + __popc(msk & lt);
-                if (pos < wcap)
-                  cand_s[static_cast<size_t>(r) * cap + qd * wcap + pos] = make_uint2(key, static_cast<uint32_t>(j));
-                else
-                  atomicOr(p.status, kStatusCandOverflow);
+            const uint32_t key = order_key(L[r]);
+            const int pos = wcnt[r] + __popc(msk & lt);
+            if (ps && pos < wcap)
+              cand_s[static_cast<size_t>(r) * cap + qd * wcap + pos] = make_uint2(key, static_cast<uint32_t>(j));
+            else if (ps)
+              atomicOr(p.status, kStatusCandOverflow);
+            wcnt[r] += __popc(msk);
+            if (ps && mode[r] == 1 && key >= base[r])
+              atomicAdd(&hs[r * kNB + hist_index(hist_bin(key, base[r], shift[r]))], 1u);
+            if (msk != 0 && mode[r] == 0) {
+              const uint32_t wmin = __reduce_min_sync(0xFFFFFFFFu, ps ? key : 0xFFFFFFFFu);
+              const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, ps ? key : 0u);
+              if (lane == 0) {
+                atomicMin(&rs[r].tmin, wmin);
+                atomicMax(&rs[r].tmax, wmax);
               }
-              wcnt[r] += __popc(msk);
-              const RowState& st = rs[r];
-              if (st.mode == 1) {
-                const uint32_t base = st.base;
-                if (ps && key >= base)
-                  atomicAdd(&hs[r * kNB + hist_index(hist_bin(key, base, st.shift))], 1u);
-              } else {
-                const uint32_t wmin = __reduce_min_sync(0xFFFFFFFFu, ps ? key : 0xFFFFFFFFu);
-                const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, ps ? key : 0u);
-                if (lane == 0) {
-                  atomicMin(&rs[r].tmin, wmin);
-                  atomicMax(&rs[r].tmax, wmax);
-                }
-                maint = true;  // the row opens its histogram window at the next vote
-              }
-              if (wcnt[r] > wcap - 64) maint = true;
+              maint = true;  // the row opens its histogram window at the next vote
             }
+            if (wcnt[r] > wcap - kVoteTiles * 32) maint = true;
           }
-          // Every other tile (and the last), one barrier carries two votes:
+          // Every kVoteTiles tiles (and the last), one barrier carries two votes:
           // abort (weight 1: lane 0 of each warp) and maintenance (weight 5:
-          // lanes 0..4 of each warp).  Between votes a warp adds at most 64
-          // candidates to its segment, which the margin above leaves room for.
-          if ((t & 1) || t + 1 == U.ntiles) {
+          // lanes 0..4 of each warp).  Between votes a warp adds at most
+          // 32 * kVoteTiles candidates to its segment, which the margin above
+          // leaves room for.
+          if ((t % kVoteTiles) == kVoteTiles - 1 || t + 1 == U.ntiles) {
             if (lane == 0) {
 #pragma unroll
               for (int r = 0; r < RW; ++r) rs[r].wcnt[qd] = min(wcnt[r], wcap);
@@ -798,7 +802,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
               for (int r = 0; r < RW; ++r) {
                 const RowState& st = rs[r];
                 opened[r] = st.mode == 0 && st.tmin != 0xFFFFFFFFu;
-                compact[r] = max(max(st.wcnt[0], st.wcnt[1]), max(st.wcnt[2], st.wcnt[3])) > wcap - 64;
+                compact[r] = max(max(st.wcnt[0], st.wcnt[1]), max(st.wcnt[2], st.wcnt[3])) > wcap - kVoteTiles * 32;
               }
               named_bar_sync(bar_id, 128);
               if (qd < RW && (compact[qd] || opened[qd])) {
@@ -858,17 +862,18 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
 #pragma unroll
               for (int r = 0; r < RW; ++r) wcnt[r] = rs[r].wcnt[qd];
             }
-            // ---- raise the threshold from the histogram (one warp per row)
-            if (qd < RW && rs[qd].mode == 1) {
-              RowState& st = rs[qd];
-              const Boundary B = find_boundary(hs + qd * kNB, static_cast<uint32_t>(k), lane);
-              if (B.found && lane == 0) {
-                uint64_t th = static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin) << st.shift);
-                if (th > 0xFFFFFFFFull) th = 0xFFFFFFFFull;
-                if (static_cast<uint32_t>(th) > st.theta) {
-                  st.theta = static_cast<uint32_t>(th);
-                  st.theta_f = theta_float(st.theta);
-                }
+          }
+          // ---- raise the threshold from the histogram: warp qd refreshes row qd
+          // every fourth tile, the warps staggered so that one refreshes per tile
+          if (qd < RW && (t & 3) == qd && rs[qd].mode == 1) {
+            RowState& st = rs[qd];
+            const Boundary B = find_boundary(hs + qd * kNB, static_cast<uint32_t>(k), lane);
+            if (B.found && lane == 0) {
+              uint64_t th = static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin) << st.shift);
+              if (th > 0xFFFFFFFFull) th = 0xFFFFFFFFull;
+              if (static_cast<uint32_t>(th) > st.theta) {
+                st.theta = static_cast<uint32_t>(th);
+                st.theta_f = theta_float(st.theta);
               }
             }
           }

@@ -14,6 +14,7 @@ constexpr int kPageSize = 64;      // tokens per key page (paged form)
 constexpr int kMaxTopK = 2048;
 constexpr int kThreads = 384;      // 12 warps: TMA, MMA, 8 epilogue, 2 select
 constexpr int kStatusBytes = 256;  // device status block at the head of every workspace
+constexpr int kVoteTiles = 8;      // tiles between the fused epilogue's group votes
 
 // device status bits (workspace word 0)
 constexpr int kStatusWaitTimeout = 1;

@@ -93,6 +93,15 @@ def test_topk_rows_exact(m, n, k):
 
 # ---------------------------------------------------------------------------- fused
 
+def _fused_call(d, k, values=True):
+    """Fused call with an explicit workspace; asserts the device status is clean."""
+    t = _to(d)
+    ws = fx.alloc_workspace(fx.mqa_logits_topk_workspace_size(d["m"], d["n"], k))
+    out = fx.mqa_logits_topk(**t, topk=k, return_values=values, workspace=ws)
+    assert fx.read_device_status(ws) == 0
+    return out
+
+
 def _check_fused(d, idx, vals, rows, k):
     ref = _oracle_rows(d, rows)
     n = d["n"]
@@ -110,8 +119,7 @@ def _check_fused(d, idx, vals, rows, k):
 def test_fused_small(m, n, k, seed):
     ks, ke = _ragged(m, n, seed)
     d = workloads.make_prefill(m, n, seed, ks=ks, ke=ke)
-    idx, vals = fx.mqa_logits_topk(**_to(d), topk=k, return_values=True)
-    torch.cuda.synchronize()
+    idx, vals = _fused_call(d, k)
     _check_fused(d, idx.cpu().numpy(), vals.cpu().numpy(), np.arange(m), k)
 
 
@@ -120,8 +128,7 @@ def test_fused_unsplit_schedule(k):
     """>= 8 x SMs rows: one unit per row block, top-k written directly."""
     m, n = 8 * fx.num_sms() + 5, 5000 if k == 2048 else 2500
     d = workloads.make_prefill(m, n, 21 + k)
-    idx, vals = fx.mqa_logits_topk(**_to(d), topk=k, return_values=True)
-    torch.cuda.synchronize()
+    idx, vals = _fused_call(d, k)
     rows = np.concatenate([np.arange(0, 8), np.arange(m - 8, m), np.arange(400, 408)])
     _check_fused(d, idx.cpu().numpy(), vals.cpu().numpy(), rows, k)
 
@@ -144,7 +151,7 @@ def test_fused_all_ties():
     """Every key identical: the top-k is the k lowest indices of each range."""
     m, n, k = 10, 3000, 256
     d = workloads.make_prefill(m, n, 5, duplicate_keys=True)
-    idx = fx.mqa_logits_topk(**_to(d), topk=k).cpu().numpy()
+    idx = _fused_call(d, k, values=False).cpu().numpy()
     for i in range(m):
         lo, hi = row_range(d["ks"][i], d["ke"][i], n)
         want = list(range(lo, min(hi, lo + k)))
@@ -198,8 +205,7 @@ def _sample_rows(m, count, seed):
 @pytest.mark.parametrize("index,count", [(0, 16), (1, 48), (2, 24), (3, 8)])
 def test_fused_full_workloads_sampled(index, count):
     d = workloads.make_workload(index)
-    idx, vals = fx.mqa_logits_topk(**_to(d), topk=workloads.TOPK, return_values=True)
-    torch.cuda.synchronize()
+    idx, vals = _fused_call(d, workloads.TOPK)
     rows = _sample_rows(d["m"], min(count, d["m"]), index)
     _check_fused(d, idx.cpu().numpy(), vals.cpu().numpy(), rows, workloads.TOPK)
 
@@ -207,7 +213,9 @@ def test_fused_full_workloads_sampled(index, count):
 def test_paged_full_workload_sampled():
     d = workloads.make_workload(4)
     t = {key: d[key].cuda() for key in ("q", "k_pages", "s_pages", "w", "block_table", "seq_lens")}
-    idx, vals = fx.paged_mqa_logits_topk(**t, R=d["R"], topk=workloads.TOPK, return_values=True)
-    torch.cuda.synchronize()
+    ws = fx.alloc_workspace(fx.paged_workspace_size(d["B"], d["R"], d["max_blocks"], workloads.TOPK))
+    idx, vals = fx.paged_mqa_logits_topk(**t, R=d["R"], topk=workloads.TOPK, return_values=True,
+                                         workspace=ws)
+    assert fx.read_device_status(ws) == 0
     rows = _sample_rows(d["B"] * d["R"], 24, 4)
     _paged_check(d, idx.cpu().numpy(), vals.cpu().numpy(), rows, workloads.TOPK)
