@@ -164,19 +164,36 @@ __device__ __forceinline__ Unit get_unit(const IndexerParams& p, int u) {
 
 // Bounded wait on an mbarrier phase.  Gives up when another role has
 // aborted or after `limit_ns`, flagging the device status; never traps.
-__device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                      int* status, unsigned long long limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+// SLEEP backs off with nanosleep (long waits of idle roles, which then take
+// no issue slots from the epilogue); otherwise it spins (latency-critical
+// hand-offs) and looks at the clock only every 64 polls.
+template <bool SLEEP>
+__device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                       int* status, unsigned long long limit_ns) {
   const uint64_t t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > limit_ns) {
-      *abort_flag = 1;
-      atomicOr(status, kStatusWaitTimeout);
-      return false;
+  uint32_t ns = 64;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (SLEEP) {
+      __nanosleep(ns);
+      if (ns < 2048) ns <<= 1;
+    }
+    if (SLEEP || (it & 63) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        atomicOr(status, kStatusWaitTimeout);
+        return false;
+      }
     }
   }
+}
+
+template <bool SLEEP>
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                           int* status, unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_slow<SLEEP>(bar, parity, abort_flag, status, limit_ns);
 }
 
 // Uniform OR over the threads of a named barrier.
@@ -207,10 +224,11 @@ __device__ __forceinline__ uint32_t bar_red_popc(int id, int nthreads, bool pred
 }
 
 // sum_h w[h] * max(x[h], 0) over the 32 heads of one (key, row), with packed
-// two-lane fp32 FMAs (each lane rounded once, like fmaf).
+// two-lane fp32 FMAs (each lane rounded once, like fmaf) into four
+// independent packed accumulators.
 __device__ __forceinline__ float relu_dot32(const uint32_t (&x)[32], const float* wsm) {
   const float4* w4 = reinterpret_cast<const float4*>(wsm);
-  uint64_t a0 = 0, a1 = 0;
+  uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 wv = w4[i];
@@ -218,13 +236,13 @@ __device__ __forceinline__ float relu_dot32(const uint32_t (&x)[32], const float
                                     fmaxf(__uint_as_float(x[4 * i + 1]), 0.f));
     const uint64_t r23 = pack_f32x2(fmaxf(__uint_as_float(x[4 * i + 2]), 0.f),
                                     fmaxf(__uint_as_float(x[4 * i + 3]), 0.f));
-    a0 = fma_f32x2(pack_f32x2(wv.x, wv.y), r01, a0);
-    a1 = fma_f32x2(pack_f32x2(wv.z, wv.w), r23, a1);
+    acc[(2 * i) & 3] = fma_f32x2(pack_f32x2(wv.x, wv.y), r01, acc[(2 * i) & 3]);
+    acc[(2 * i + 1) & 3] = fma_f32x2(pack_f32x2(wv.z, wv.w), r23, acc[(2 * i + 1) & 3]);
   }
-  float s0, s1, s2, s3;
-  unpack_f32x2(a0, s0, s1);
-  unpack_f32x2(a1, s2, s3);
-  return (s0 + s1) + (s2 + s3);
+  float s[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) unpack_f32x2(acc[i], s[2 * i], s[2 * i + 1]);
+  return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
 }
 
 // Histogram slot of bin b: lane (b >> 4) owns bins [16 lane, 16 lane + 16),
@@ -437,8 +455,9 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
   constexpr int S = C::STAGES;
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base (128-byte swizzled TMA tiles), derived by pointer
+  // arithmetic on the shared array so that accesses stay shared-memory ones
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* q_smem = smem + SL.q;
   uint8_t* stage_smem = smem + SL.stage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL.bar);
@@ -511,13 +530,13 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         const int u = p.num_units - 1 - i;
         const Unit U = get_unit<R, PAGED>(p, u);
         if (U.ntiles == 0) continue;
-        if (!wait_bar(qempty, qphase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
+        if (!wait_phase<true>(qempty, qphase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
         qphase ^= 1;
         mbar_arrive_expect_tx(qfull, C::Q_BYTES);
         tma_load_2d(q_smem, &p.tmap_q, qfull, 0, U.row0 * kHeads);
         const int32_t* bt = PAGED ? p.block_table + static_cast<int64_t>(U.req) * p.max_blocks : nullptr;
         for (int t = 0; t < U.ntiles; ++t) {
-          if (!wait_bar(&empty[stage], phase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
+          if (!wait_phase<true>(&empty[stage], phase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
           const int j0 = U.jbeg + t * kBlockKeys;
           uint8_t* dst = stage_smem + stage * C::TILE_BYTES;
           if (!PAGED) {
@@ -565,15 +584,15 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         const int u = p.num_units - 1 - i;
         const Unit U = get_unit<R, PAGED>(p, u);
         if (U.ntiles == 0) continue;
-        if (!wait_bar(qfull, qphase, abort_flag, p.status, limit)) { ok = false; break; }
+        if (!wait_phase<false>(qfull, qphase, abort_flag, p.status, limit)) { ok = false; break; }
         qphase ^= 1;
         tc_fence_after();
         const uint64_t bdesc = smem_desc_k128_sw128(q_addr);
         for (int t = 0; t < U.ntiles; ++t, ++T) {
           const uint32_t a = T & 1, aph = (T >> 1) & 1;
-          if (!wait_bar(&tempty[a], aph ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
+          if (!wait_phase<false>(&tempty[a], aph ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
           tc_fence_after();
-          if (!wait_bar(&full[stage], phase, abort_flag, p.status, limit)) { ok = false; break; }
+          if (!wait_phase<false>(&full[stage], phase, abort_flag, p.status, limit)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = smem_desc_k128_sw128(smem_u32(stage_smem + stage * C::TILE_BYTES));
           const uint32_t d = tbase + a * N;
@@ -624,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
                           ? p.cand + (static_cast<size_t>(blockIdx.x * 2 + slot) * R + g * RW) * cap
                           : nullptr;
       if (MODE == kModeTopK) {
-        if (!wait_bar(&slot_empty[slot], ((it >> 1) & 1) ^ 1, abort_flag, p.status, limit)) aborted = true;
+        if (!wait_phase<true>(&slot_empty[slot], ((it >> 1) & 1) ^ 1, abort_flag, p.status, limit)) aborted = true;
       }
       // ---- per-row setup for this warpgroup's rows: the key range [lo, hi)
       // (kept in shared memory; the tile loop reads it back as a broadcast)
@@ -710,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         const float sj = s_next;
         if (t + 1 < U.ntiles) s_next = scale_of(j + kBlockKeys);
         const uint32_t a = T & 1, aph = (T >> 1) & 1;
-        if (!wait_bar(&tfull[a], aph, abort_flag, p.status, limit)) aborted = true;
+        if (!wait_phase<false>(&tfull[a], aph, abort_flag, p.status, limit)) aborted = true;
         tc_fence_after();
         float L[RW];
 #pragma unroll
@@ -754,22 +773,33 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
             base[r] = st.base;
             shift[r] = st.shift;
           }
+          bool ps[RW];
+          uint32_t msk[RW], key[RW];
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
-            const bool ps = j >= lo[r] && j < hi[r] && L[r] >= thf[r];
-            const uint32_t msk = __ballot_sync(0xFFFFFFFFu, ps);
-            const uint32_t key = order_key(L[r]);
-            const int pos = wcnt[r] + __popc(msk & lt);
-            if (ps && pos < wcap)
-              cand_s[static_cast<size_t>(r) * cap + qd * wcap + pos] = make_uint2(key, static_cast<uint32_t>(j));
-            else if (ps)
+            ps[r] = j >= lo[r] && j < hi[r] && L[r] >= thf[r];
+            msk[r] = __ballot_sync(0xFFFFFFFFu, ps[r]);
+            key[r] = order_key(L[r]);
+          }
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            const int pos = wcnt[r] + __popc(msk[r] & lt);
+            wcnt[r] += __popc(msk[r]);
+            if (ps[r] && pos < wcap)
+              cand_s[static_cast<size_t>(r) * cap + qd * wcap + pos] = make_uint2(key[r], static_cast<uint32_t>(j));
+            else if (ps[r])
               atomicOr(p.status, kStatusCandOverflow);
-            wcnt[r] += __popc(msk);
-            if (ps && mode[r] == 1 && key >= base[r])
-              atomicAdd(&hs[r * kNB + hist_index(hist_bin(key, base[r], shift[r]))], 1u);
-            if (msk != 0 && mode[r] == 0) {
-              const uint32_t wmin = __reduce_min_sync(0xFFFFFFFFu, ps ? key : 0xFFFFFFFFu);
-              const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, ps ? key : 0u);
+          }
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            if (ps[r] && mode[r] == 1 && key[r] >= base[r])
+              atomicAdd(&hs[r * kNB + hist_index(hist_bin(key[r], base[r], shift[r]))], 1u);
+          }
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            if (msk[r] != 0 && mode[r] == 0) {
+              const uint32_t wmin = __reduce_min_sync(0xFFFFFFFFu, ps[r] ? key[r] : 0xFFFFFFFFu);
+              const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, ps[r] ? key[r] : 0u);
               if (lane == 0) {
                 atomicMin(&rs[r].tmin, wmin);
                 atomicMax(&rs[r].tmax, wmax);
@@ -901,7 +931,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
     const int wcap = cap >> 2;
     for (int i = blockIdx.x, it = 0; i < p.num_units; i += gridDim.x, ++it) {
       const int slot = it & 1;
-      const bool ok = wait_bar(&slot_full[slot], (it >> 1) & 1, abort_flag, p.status, limit);
+      const bool ok = wait_phase<true>(&slot_full[slot], (it >> 1) & 1, abort_flag, p.status, limit);
       if (bar_red_or(kSelBar, NT, !ok || *abort_flag)) break;
       const SlotMeta meta = smeta[slot];
       for (int rl = 0; rl < R; ++rl) {
