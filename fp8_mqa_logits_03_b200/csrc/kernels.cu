@@ -249,6 +249,7 @@ __device__ __forceinline__ float relu_dot32(const uint32_t (&x)[32], const float
 // stored transposed so that a warp reading one bin per lane hits 32 banks.
 __device__ __forceinline__ int hist_index(int b) { return (b & 15) * 32 + (b >> 4); }
 
+// (Only meaningful for key >= base; any other key maps to some bin in range.)
 __device__ __forceinline__ int hist_bin(uint32_t key, uint32_t base, int shift) {
   return static_cast<int>(min((key - base) >> shift, static_cast<uint32_t>(kNB - 1)));
 }
@@ -280,20 +281,20 @@ __device__ __forceinline__ Boundary find_boundary(const uint32_t* h, uint32_t k,
   const uint32_t ball = __ballot_sync(0xFFFFFFFFu, suf >= k);
   if (ball == 0) return B;
   const int ls = 31 - __clz(static_cast<int>(ball));
+  // inside lane ls: the highest of its 16 bins where the running count from
+  // the top reaches k (predicated, no divergent loop)
+  uint32_t run = suf - tot;
   int bin = 0;
   uint32_t above = 0, inbin = 0;
-  if (lane == ls) {
-    uint32_t run = suf - tot;
+  bool done = false;
 #pragma unroll
-    for (int i = 15; i >= 0; --i) {
-      if (run + c[i] >= k) {
-        bin = ls * 16 + i;
-        inbin = c[i];
-        break;
-      }
-      run += c[i];
-    }
-    above = run;
+  for (int i = 15; i >= 0; --i) {
+    const bool hit = !done && run + c[i] >= k;
+    bin = hit ? lane * 16 + i : bin;
+    inbin = hit ? c[i] : inbin;
+    above = hit ? run : above;
+    done = done || hit;
+    run += c[i];
   }
   B.found = true;
   B.bin = __shfl_sync(0xFFFFFFFFu, bin, ls);
@@ -723,7 +724,6 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         return __ldg(p.s + static_cast<int64_t>(pg) * kPageSize + (j % kPageSize));
       };
       float s_next = U.ntiles ? scale_of(key0) : 0.f;
-      bool maint = false;  // this warp saw a row that needs maintenance at the next vote
       for (int t = 0; t < U.ntiles; ++t, ++T) {
         const int j = key0 + t * kBlockKeys;
         const float sj = s_next;
@@ -773,54 +773,35 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
             base[r] = st.base;
             shift[r] = st.shift;
           }
-          bool ps[RW];
-          uint32_t msk[RW], key[RW];
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
-            ps[r] = j >= lo[r] && j < hi[r] && L[r] >= thf[r];
-            msk[r] = __ballot_sync(0xFFFFFFFFu, ps[r]);
-            key[r] = order_key(L[r]);
-          }
-#pragma unroll
-          for (int r = 0; r < RW; ++r) {
-            const int pos = wcnt[r] + __popc(msk[r] & lt);
-            wcnt[r] += __popc(msk[r]);
-            if (ps[r] && pos < wcap)
-              cand_s[static_cast<size_t>(r) * cap + qd * wcap + pos] = make_uint2(key[r], static_cast<uint32_t>(j));
-            else if (ps[r])
-              atomicOr(p.status, kStatusCandOverflow);
-          }
-#pragma unroll
-          for (int r = 0; r < RW; ++r) {
-            if (ps[r] && mode[r] == 1 && key[r] >= base[r])
-              atomicAdd(&hs[r * kNB + hist_index(hist_bin(key[r], base[r], shift[r]))], 1u);
-          }
-#pragma unroll
-          for (int r = 0; r < RW; ++r) {
-            if (msk[r] != 0 && mode[r] == 0) {
-              const uint32_t wmin = __reduce_min_sync(0xFFFFFFFFu, ps[r] ? key[r] : 0xFFFFFFFFu);
-              const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, ps[r] ? key[r] : 0u);
-              if (lane == 0) {
-                atomicMin(&rs[r].tmin, wmin);
-                atomicMax(&rs[r].tmax, wmax);
-              }
-              maint = true;  // the row opens its histogram window at the next vote
-            }
-            if (wcnt[r] > wcap - kVoteTiles * 32) maint = true;
+            const bool ps = j >= lo[r] && j < hi[r] && L[r] >= thf[r];
+            const uint32_t msk = __ballot_sync(0xFFFFFFFFu, ps);
+            const uint32_t key = order_key(L[r]);
+            const int pos = wcnt[r] + __popc(msk & lt);
+            wcnt[r] += __popc(msk);
+            uint2* dst = cand_s + (r * cap + qd * wcap + min(pos, wcap - 1));
+            if (ps && pos < wcap) *dst = make_uint2(key, static_cast<uint32_t>(j));
+            const int hidx = r * kNB + hist_index(hist_bin(key, base[r], shift[r]));
+            if (ps && mode[r] == 1 && key >= base[r]) atomicAdd(&hs[hidx], 1u);
           }
           // Every kVoteTiles tiles (and the last), one barrier carries two votes:
           // abort (weight 1: lane 0 of each warp) and maintenance (weight 5:
-          // lanes 0..4 of each warp).  Between votes a warp adds at most
-          // 32 * kVoteTiles candidates to its segment, which the margin above
-          // leaves room for.
+          // lanes 0..4 of each warp): a row still without its histogram window
+          // has candidates, or a segment is within 32 * kVoteTiles of full.
           if ((t % kVoteTiles) == kVoteTiles - 1 || t + 1 == U.ntiles) {
+            bool maint = false;
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+              maint |= (mode[r] == 0 && wcnt[r] > 0) || wcnt[r] > wcap - kVoteTiles * 32;
+              if (wcnt[r] > wcap && lane == 0) atomicOr(p.status, kStatusCandOverflow);
+            }
             if (lane == 0) {
 #pragma unroll
               for (int r = 0; r < RW; ++r) rs[r].wcnt[qd] = min(wcnt[r], wcap);
             }
             const bool ab = aborted || *abort_flag;
             const uint32_t votes = bar_red_popc(bar_id, 128, (lane == 0 && ab) || (lane < 5 && maint));
-            maint = false;
             if (votes % 5) {
               aborted = true;
               break;
@@ -831,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
 #pragma unroll
               for (int r = 0; r < RW; ++r) {
                 const RowState& st = rs[r];
-                opened[r] = st.mode == 0 && st.tmin != 0xFFFFFFFFu;
+                opened[r] = st.mode == 0 && (st.wcnt[0] + st.wcnt[1] + st.wcnt[2] + st.wcnt[3]) > 0;
                 compact[r] = max(max(st.wcnt[0], st.wcnt[1]), max(st.wcnt[2], st.wcnt[3])) > wcap - kVoteTiles * 32;
               }
               named_bar_sync(bar_id, 128);
@@ -839,15 +820,36 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
                 RowState& st = rs[qd];
                 uint2* rowbuf = cand_s + static_cast<size_t>(qd) * cap;
                 uint32_t* h = hs + qd * kNB;
-                if (opened[qd] && lane == 0) {
-                  // window over twice the span of the keys collected so far
-                  const uint64_t span = static_cast<uint64_t>(st.tmax - st.tmin);
+                if (opened[qd]) {
+                  // Open the row's histogram window over twice the span of the keys
+                  // collected so far (at most kVoteTiles tiles' worth) and count them.
+                  uint32_t kmin = 0xFFFFFFFFu, kmax = 0;
+                  for (int s = 0; s < 4; ++s)
+                    for (int e = lane; e < st.wcnt[s]; e += 32) {
+                      const uint32_t key = rowbuf[s * wcap + e].x;
+                      kmin = min(kmin, key);
+                      kmax = max(kmax, key);
+                    }
+                  kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+                  kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+                  const uint64_t span = static_cast<uint64_t>(kmax - kmin);
                   const int bits = 64 - __clzll(static_cast<long long>(2 * span + 1));
-                  st.base = st.tmin;
-                  st.shift = bits > 9 ? bits - 9 : 0;
-                  st.mode = 1;
+                  const uint32_t wbase = kmin;
+                  const int wshift = bits > 9 ? bits - 9 : 0;
+                  if (!compact[qd])
+                    for (int s = 0; s < 4; ++s)
+                      for (int e = lane; e < st.wcnt[s]; e += 32) {
+                        const uint32_t key = rowbuf[s * wcap + e].x;
+                        atomicAdd(&h[hist_index(hist_bin(key, wbase, wshift))], 1u);
+                      }
+                  __syncwarp();
+                  if (lane == 0) {
+                    st.base = wbase;
+                    st.shift = wshift;
+                    st.mode = 1;
+                  }
+                  __syncwarp();
                 }
-                __syncwarp();
                 if (compact[qd]) {
                   // Rare: a segment is near full.  Keep the row's exact top-k (later keys
                   // have larger indices, so a key equal to the k-th value never enters
@@ -876,15 +878,6 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
                   for (int e = lane; e < kept; e += 32) {
                     const uint32_t key = scr[e].x;
                     if (key >= st.base) atomicAdd(&h[hist_index(hist_bin(key, st.base, st.shift))], 1u);
-                  }
-                } else {
-                  // count the few candidates collected before the window opened
-                  for (int s = 0; s < 4; ++s) {
-                    const uint2* seg = rowbuf + s * wcap;
-                    for (int e = lane; e < st.wcnt[s]; e += 32) {
-                      const uint32_t key = seg[e].x;
-                      if (key >= st.base) atomicAdd(&h[hist_index(hist_bin(key, st.base, st.shift))], 1u);
-                    }
                   }
                 }
               }
