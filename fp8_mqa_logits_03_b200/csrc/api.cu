@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "../../include/fp8idx.h"
@@ -16,6 +17,14 @@
 
 namespace fp8idx {
 __device__ int g_logits_status;  // device status of the last fp8idx_mqa_logits call
+
+// Fixed scratch of fp8idx_mqa_logits_topk_noalloc: a module-scope device
+// array, so it is created when the library's device code is loaded on a GPU
+// and lives until the process exits (64 MiB on every GPU that loads it).
+// On the host this name is only a stand-in for the device symbol; its device
+// address comes from cudaGetSymbolAddress.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 }
 
 namespace {
@@ -427,6 +436,102 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
   if (e != cudaSuccess) return cuda_fail(e, "paged_mqa_logits_topk launch");
   if (pl.n_chunks > 1) {
     MergeParams mp{p.part, p.part_cnt, static_cast<int>(B * R), pl.R, pl.n_chunks, topk, out_idx, out_vals};
+    e = launch_merge(mp, st);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  }
+  return ok();
+}
+
+// Allocation-free form of fp8idx_mqa_logits_topk for callers that cannot
+// allocate device memory at call time: code running while a CUDA graph is
+// captured or replayed by a framework that owns every allocation, inference
+// runtimes with a fixed memory budget planned at start-up, or plugins whose
+// host forbids cudaMalloc outside initialisation.  The workspace is the fixed
+// array above instead of a caller buffer.  The first call on each device
+// looks up the array's device address (once, under a lock); make that first
+// call before capturing a stream.  The grid shrinks until the workspace plan
+// fits in the array, so large problems run on fewer SMs (slower, same
+// result); a problem that does not fit even on one SM is rejected with
+// FP8IDX_EWORKSPACE.  Every call reuses the same array, which keeps the last
+// call's contents; the status block is cleared on entry.  Two calls that may
+// run at the same time on the GPU (different streams, or different host
+// threads) race on the array and must be serialised by the caller.
+int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const float* s,
+                                   const float* w, const int32_t* ks, const int32_t* ke, int64_t m,
+                                   int64_t n, int H, int D, int topk, int32_t* out_idx,
+                                   float* out_vals, void* stream) {
+  FP8IDX_TRY(check_shape(H, D));
+  FP8IDX_TRY(check_topk(topk));
+  FP8IDX_TRY(check_prefill_inputs(q, k, s, w, ks, ke, m, n));
+  if (m == 0) return ok();
+  if (!out_idx || !aligned(out_idx, 4) || !aligned(out_vals, 4))
+    return fail(FP8IDX_EINVAL, "out_idx must be non-null; outputs 4-byte aligned");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "current device");
+  constexpr int kMaxDevices = 64;
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP8IDX_EUNSUPPORTED, "device index %d out of range", dev);
+  static std::mutex mu;
+  static void* scratch_of[kMaxDevices] = {};
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!scratch_of[dev]) {
+      void* ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "no-alloc scratch address");
+      scratch_of[dev] = ptr;
+    }
+    scratch = scratch_of[dev];
+  }
+  int sms = device_sms();
+  if (sms <= 0) return fail(FP8IDX_ECUDA, "no CUDA device");
+  Plan pl;
+  int g = sms;
+  for (; g >= 1; --g) {
+    pl = plan_prefill(m, n, topk, g);
+    if (pl.total <= kNoAllocScratchBytes) break;
+  }
+  if (g < 1)
+    return fail(FP8IDX_EWORKSPACE, "problem needs more than the %zu-byte fixed scratch", kNoAllocScratchBytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(scratch);
+  e = cudaMemsetAsync(wsb, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+  if (n == 0) {
+    e = launch_fill_empty(out_idx, out_vals, static_cast<int>(m), topk, st);
+    if (e != cudaSuccess) return cuda_fail(e, "fill launch");
+    return ok();
+  }
+  IndexerParams p;
+  memset(&p, 0, sizeof(p));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, m * kHeads, pl.R * kHeads));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_k, k, n, kBlockKeys));
+  p.s = s;
+  p.w = w;
+  p.ks = ks;
+  p.ke = ke;
+  p.n = n;
+  p.m = static_cast<int>(m);
+  p.topk = topk;
+  p.n_chunks = pl.n_chunks;
+  p.chunk_keys = pl.chunk_keys;
+  p.num_units = pl.num_units;
+  p.out_idx = out_idx;
+  p.out_vals = out_vals;
+  p.status = reinterpret_cast<int*>(wsb);
+  p.cand = reinterpret_cast<uint2*>(wsb + pl.off_cand);
+  p.cand_cap = pl.cap;
+  p.scratch = reinterpret_cast<uint2*>(wsb + pl.off_scratch);
+  if (pl.n_chunks > 1) {
+    p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
+    p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
+  }
+  p.wait_limit_ns = g_wait_limit_ns;
+  e = launch_indexer_prefill_topk(p, pl.grid, st);
+  if (e != cudaSuccess) return cuda_fail(e, "mqa_logits_topk_noalloc launch");
+  if (pl.n_chunks > 1) {
+    MergeParams mp{p.part, p.part_cnt, static_cast<int>(m), pl.R, pl.n_chunks, topk, out_idx, out_vals};
     e = launch_merge(mp, st);
     if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }

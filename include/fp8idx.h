@@ -136,6 +136,26 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
                                  void* stream);
 
 /*
+ * Allocation-free variant of fp8idx_mqa_logits_topk (the pages have no
+ * counterpart: it exists for callers that cannot allocate device memory at
+ * call time, such as code inside a framework-owned CUDA graph or a runtime
+ * with a fixed, pre-planned memory budget).  Same arguments and result as
+ * fp8idx_mqa_logits_topk without ws / ws_bytes: the library keeps a fixed
+ * 64 MiB device array as its workspace, created when the library's device
+ * code loads on a GPU and held until the process exits.  The first call on a
+ * device looks up that array's address; make it before any stream capture.
+ * Large problems run on fewer SMs so that the workspace fits; a problem that
+ * does not fit at all returns FP8IDX_EWORKSPACE.  All calls share the array:
+ * calls that can overlap on the GPU race and must be serialised by the
+ * caller.  The device status of the last call is not readable through this
+ * entry point's interface.
+ */
+int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const float* s,
+                                   const float* w, const int32_t* ks, const int32_t* ke, int64_t m,
+                                   int64_t n, int H, int D, int topk, int32_t* out_idx,
+                                   float* out_vals, void* stream);
+
+/*
  * Tests and diagnostics.  fp8idx_read_device_status synchronises `stream`
  * and copies the status word written by the last call that used workspace
  * `ws` (ws == NULL: the last fp8idx_mqa_logits call) into *status_out.
