@@ -223,26 +223,32 @@ __device__ __forceinline__ uint32_t bar_red_popc(int id, int nthreads, bool pred
   return r;
 }
 
-// sum_h w[h] * max(x[h], 0) over the 32 heads of one (key, row), with packed
-// two-lane fp32 FMAs (each lane rounded once, like fmaf) into four
-// independent packed accumulators.
-__device__ __forceinline__ float relu_dot32(const uint32_t (&x)[32], const float* wsm) {
+// 2 * sum_h w[h] * max(x[h], 0) over the 32 heads of one (key, row), as
+// sum_h (w[h] * x[h] + w[h] * |x[h]|): the identity 2 max(x, 0) = x + |x| keeps
+// the whole reduction on the FMA pipe (|x| is a free operand modifier) and off
+// the half-rate min/max pipe.  The linear half uses packed two-lane FMAs.
+// Each FMA rounds once; the extra rounding against the max form is a few
+// units in the last place of the running sum.  Callers scale by 0.5.
+__device__ __forceinline__ float relu_dot32_x2(const uint32_t (&x)[32], const float* wsm) {
   const float4* w4 = reinterpret_cast<const float4*>(wsm);
-  uint64_t acc[4] = {0, 0, 0, 0};
+  uint64_t lin0 = 0, lin1 = 0;
+  float ab0 = 0.f, ab1 = 0.f, ab2 = 0.f, ab3 = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 wv = w4[i];
-    const uint64_t r01 = pack_f32x2(fmaxf(__uint_as_float(x[4 * i + 0]), 0.f),
-                                    fmaxf(__uint_as_float(x[4 * i + 1]), 0.f));
-    const uint64_t r23 = pack_f32x2(fmaxf(__uint_as_float(x[4 * i + 2]), 0.f),
-                                    fmaxf(__uint_as_float(x[4 * i + 3]), 0.f));
-    acc[(2 * i) & 3] = fma_f32x2(pack_f32x2(wv.x, wv.y), r01, acc[(2 * i) & 3]);
-    acc[(2 * i + 1) & 3] = fma_f32x2(pack_f32x2(wv.z, wv.w), r23, acc[(2 * i + 1) & 3]);
+    const float x0 = __uint_as_float(x[4 * i + 0]), x1 = __uint_as_float(x[4 * i + 1]);
+    const float x2 = __uint_as_float(x[4 * i + 2]), x3 = __uint_as_float(x[4 * i + 3]);
+    lin0 = fma_f32x2(pack_f32x2(wv.x, wv.y), pack_f32x2(x0, x1), lin0);
+    lin1 = fma_f32x2(pack_f32x2(wv.z, wv.w), pack_f32x2(x2, x3), lin1);
+    ab0 = fmaf(wv.x, fabsf(x0), ab0);
+    ab1 = fmaf(wv.y, fabsf(x1), ab1);
+    ab2 = fmaf(wv.z, fabsf(x2), ab2);
+    ab3 = fmaf(wv.w, fabsf(x3), ab3);
   }
-  float s[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) unpack_f32x2(acc[i], s[2 * i], s[2 * i + 1]);
-  return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+  float l0, l1, l2, l3;
+  unpack_f32x2(lin0, l0, l1);
+  unpack_f32x2(lin1, l2, l3);
+  return ((l0 + ab0) + (l1 + ab1)) + ((l2 + ab2) + (l3 + ab3));
 }
 
 // Histogram slot of bin b: lane (b >> 4) owns bins [16 lane, 16 lane + 16),
@@ -726,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       float s_next = U.ntiles ? scale_of(key0) : 0.f;
       for (int t = 0; t < U.ntiles; ++t, ++T) {
         const int j = key0 + t * kBlockKeys;
-        const float sj = s_next;
+        const float sj = 0.5f * s_next;  // relu_dot32_x2 returns twice the head sum
         if (t + 1 < U.ntiles) s_next = scale_of(j + kBlockKeys);
         const uint32_t a = T & 1, aph = (T >> 1) & 1;
         if (!wait_phase<false>(&tfull[a], aph, abort_flag, p.status, limit)) aborted = true;
@@ -743,8 +749,8 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[a]);
           }
-          L[r] = relu_dot32(x0, ws_g + r * kHeads) * sj;
-          L[r + 1] = relu_dot32(x1, ws_g + (r + 1) * kHeads) * sj;
+          L[r] = relu_dot32_x2(x0, ws_g + r * kHeads) * sj;
+          L[r + 1] = relu_dot32_x2(x1, ws_g + (r + 1) * kHeads) * sj;
         }
 
         if (MODE == kModeLogits) {
