@@ -48,8 +48,7 @@ struct Cfg {
   static constexpr int Q_BYTES = N * kDim;
   static constexpr int TILE_BYTES = kBlockKeys * kDim;
   static constexpr int TMEM_COLS = 2 * N;
-  static constexpr int NH = N / 2;              // columns of one epilogue warpgroup's half
-  static constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockKeys, NH);
+  static constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockKeys, N);
   static_assert(N <= 256 && N % 16 == 0, "MMA N out of range");
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns must be a power of two");
 };
@@ -97,7 +96,7 @@ __host__ __device__ constexpr SmemLayout smem_layout() {
   L.q = 0;
   L.stage = C::Q_BYTES;
   L.bar = L.stage + C::STAGES * C::TILE_BYTES;
-  L.misc = L.bar + 8 * (2 * C::STAGES + 16);
+  L.misc = L.bar + 8 * (2 * C::STAGES + 12);
   L.w = L.misc + 64;
   L.rows = L.w + R * kHeads * 4;
   L.meta = L.rows + 2 * R * static_cast<int>(sizeof(RowState));
@@ -458,6 +457,7 @@ template <int R, bool PAGED, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_constant__ IndexerParams p) {
   using C = Cfg<R, PAGED>;
   constexpr SmemLayout SL = smem_layout<R, PAGED>();
+  constexpr int N = C::N;
   constexpr int RW = C::RW;
   constexpr int S = C::STAGES;
 
@@ -470,13 +470,13 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL.bar);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
-  uint64_t* tfull = bars + 2 * S;       // [half][buffer]
-  uint64_t* tempty = bars + 2 * S + 4;  // [half][buffer]
-  uint64_t* qfull = bars + 2 * S + 8;
-  uint64_t* qempty = bars + 2 * S + 9;
-  uint64_t* drain = bars + 2 * S + 10;
-  uint64_t* slot_full = bars + 2 * S + 11;
-  uint64_t* slot_empty = bars + 2 * S + 13;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* qfull = bars + 2 * S + 4;
+  uint64_t* qempty = bars + 2 * S + 5;
+  uint64_t* drain = bars + 2 * S + 6;
+  uint64_t* slot_full = bars + 2 * S + 7;
+  uint64_t* slot_empty = bars + 2 * S + 9;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SL.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL.misc + 4);
   float* w_smem = reinterpret_cast<float*>(smem + SL.w);
@@ -494,18 +494,16 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 2);  // released by both halves' MMAs
-    }
-    for (int x = 0; x < 4; ++x) {
-      mbar_init(&tfull[x], 1);
-      mbar_init(&tempty[x], 4);  // the four warps of one epilogue warpgroup
+      mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);
       mbar_init(&slot_full[a], 8);
       mbar_init(&slot_empty[a], kSelWarps);
     }
     mbar_init(qfull, 1);
-    mbar_init(qempty, 2);
+    mbar_init(qempty, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -582,92 +580,41 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    // Two independent streams over the same (unit, tile) sequence, one per
-    // epilogue warpgroup: stream h multiplies each key tile by the q rows of
-    // warpgroup h (N = R/2 * 32 columns) into its own double-buffered TMEM
-    // accumulator.  A stream issues whenever its stage is loaded and its
-    // accumulator is free, so one warpgroup can run ahead of the other by up
-    // to the depth of the stage ring.
     if (lane == 0) {
-      struct Stream {
-        int i, t, stage, ntiles;
-        uint32_t phase, qphase, T;
-        bool in_unit, done;
-      };
-      Stream st[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) st[h] = Stream{static_cast<int>(blockIdx.x), 0, 0, 0, 0u, 0u, 0u, false, false};
+      int stage = 0;
+      uint32_t phase = 0, qphase = 0;
+      uint32_t T = 0;
+      bool ok = true;
+      bool any = false;
       const uint32_t q_addr = smem_u32(q_smem);
-      bool any = false, failed = false;
-      const uint64_t t_start = global_timer_ns();
-      uint64_t t_idle = t_start;
-      uint32_t polls = 0;
-      while (!(st[0].done && st[1].done) && !failed) {
-        bool progressed = false;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          Stream& S_ = st[h];
-          if (S_.done) continue;
-          if (!S_.in_unit) {
-            while (S_.i < p.num_units) {  // next unit that has tiles
-              const Unit U = get_unit<R, PAGED>(p, p.num_units - 1 - S_.i);
-              if (U.ntiles > 0) {
-                S_.ntiles = U.ntiles;
-                break;
-              }
-              S_.i += gridDim.x;
-            }
-            if (S_.i >= p.num_units) {
-              S_.done = true;
-              continue;
-            }
-            if (!mbar_try_wait(qfull, S_.qphase)) continue;
-            S_.qphase ^= 1;
-            S_.in_unit = true;
-            S_.t = 0;
-            tc_fence_after();
-          }
-          const uint32_t a = S_.T & 1, aph = (S_.T >> 1) & 1;
-          if (!mbar_try_wait(&tempty[2 * h + a], aph ^ 1)) continue;
-          if (!mbar_try_wait(&full[S_.stage], S_.phase)) continue;
+      for (int i = blockIdx.x; ok && i < p.num_units; i += gridDim.x) {
+        const int u = p.num_units - 1 - i;
+        const Unit U = get_unit<R, PAGED>(p, u);
+        if (U.ntiles == 0) continue;
+        if (!wait_phase<false>(qfull, qphase, abort_flag, p.status, limit)) { ok = false; break; }
+        qphase ^= 1;
+        tc_fence_after();
+        const uint64_t bdesc = smem_desc_k128_sw128(q_addr);
+        for (int t = 0; t < U.ntiles; ++t, ++T) {
+          const uint32_t a = T & 1, aph = (T >> 1) & 1;
+          if (!wait_phase<false>(&tempty[a], aph ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t adesc = smem_desc_k128_sw128(smem_u32(stage_smem + S_.stage * C::TILE_BYTES));
-          const uint64_t bdesc = smem_desc_k128_sw128(q_addr + h * C::NH * kDim);
-          const uint32_t d = tbase + (2 * h + a) * C::NH;
+          if (!wait_phase<false>(&full[stage], phase, abort_flag, p.status, limit)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_k128_sw128(smem_u32(stage_smem + stage * C::TILE_BYTES));
+          const uint32_t d = tbase + a * N;
 #pragma unroll
           for (int kk = 0; kk < kDim / 32; ++kk)
             mma_f8(d, adesc + 2 * kk, bdesc + 2 * kk, C::IDESC, kk > 0 ? 1u : 0u);
-          mma_commit(&empty[S_.stage]);
-          mma_commit(&tfull[2 * h + a]);
+          mma_commit(&empty[stage]);
+          mma_commit(&tfull[a]);
           any = true;
-          progressed = true;
-          ++S_.T;
-          if (++S_.stage == S) {
-            S_.stage = 0;
-            S_.phase ^= 1;
-          }
-          if (++S_.t == S_.ntiles) {
-            mma_commit(qempty);
-            S_.in_unit = false;
-            S_.i += gridDim.x;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
           }
         }
-        if (progressed) {
-          t_idle = 0;
-          polls = 0;
-          continue;
-        }
-        __nanosleep(20);  // nothing ready: yield the issue slot briefly
-        if ((++polls & 63) == 0) {
-          const uint64_t now = global_timer_ns();
-          if (t_idle == 0) t_idle = now;
-          if (*abort_flag) failed = true;
-          if (now - t_idle > limit) {
-            *abort_flag = 1;
-            atomicOr(p.status, kStatusWaitTimeout);
-            failed = true;
-          }
-        }
+        if (ok) mma_commit(qempty);
       }
       if (any) {  // all MMAs retired before TMEM is released
         mma_commit(drain);
@@ -788,19 +735,19 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         const float sj = 0.5f * s_next;  // relu_dot32_x2 returns twice the head sum
         if (t + 1 < U.ntiles) s_next = scale_of(j + kBlockKeys);
         const uint32_t a = T & 1, aph = (T >> 1) & 1;
-        if (!wait_phase<false>(&tfull[2 * g + a], aph, abort_flag, p.status, limit)) aborted = true;
+        if (!wait_phase<false>(&tfull[a], aph, abort_flag, p.status, limit)) aborted = true;
         tc_fence_after();
         float L[RW];
 #pragma unroll
         for (int r = 0; r < RW; r += 2) {  // two rows (64 columns) per TMEM read
           uint32_t x0[32], x1[32];
-          tmem_ld32(lane_addr + (2 * g + a) * C::NH + r * kHeads, x0);
-          tmem_ld32(lane_addr + (2 * g + a) * C::NH + (r + 1) * kHeads, x1);
+          tmem_ld32(lane_addr + a * N + (g * RW + r) * kHeads, x0);
+          tmem_ld32(lane_addr + a * N + (g * RW + r + 1) * kHeads, x1);
           tmem_ld_wait();
           if (r + 2 == RW) {  // the accumulator is in registers now
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[2 * g + a]);
+            if (lane == 0) mbar_arrive(&tempty[a]);
           }
           L[r] = relu_dot32_x2(x0, ws_g + r * kHeads) * sj;
           L[r + 1] = relu_dot32_x2(x1, ws_g + (r + 1) * kHeads) * sj;
