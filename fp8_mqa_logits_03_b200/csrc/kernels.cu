@@ -715,10 +715,22 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         }
       }
 
-      // ---- this warp's segment counts (reloaded after maintenance)
+      // ---- this warp's segment counts (reloaded after maintenance), its segment
+      // of each row's buffer, and the row state it reads once per vote period
       int wcnt[RW];
+      uint2* seg[RW];
+      int lo[RW], span[RW], mode[RW], shift[RW];
+      uint32_t base[RW];
 #pragma unroll
-      for (int r = 0; r < RW; ++r) wcnt[r] = 0;
+      for (int r = 0; r < RW; ++r) {
+        wcnt[r] = 0;
+        seg[r] = MODE == kModeTopK ? cand_s + static_cast<size_t>(r) * cap + qd * wcap : nullptr;
+        lo[r] = rs[r].lo;
+        span[r] = rs[r].hi - rs[r].lo;
+        mode[r] = 0;
+        shift[r] = 0;
+        base[r] = 0;
+      }
 
       // ---- stream the unit's key tiles
       const int key0 = U.jbeg + qd * 32 + lane;
@@ -766,28 +778,17 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
           }
         } else {
           // ---- filter against the running threshold; append to this warp's segment
-          int lo[RW], hi[RW], mode[RW], shift[RW];
-          uint32_t base[RW];
           float thf[RW];
 #pragma unroll
-          for (int r = 0; r < RW; ++r) {  // row state, read once per tile
-            const RowState& st = rs[r];
-            lo[r] = st.lo;
-            hi[r] = st.hi;
-            thf[r] = st.theta_f;
-            mode[r] = st.mode;
-            base[r] = st.base;
-            shift[r] = st.shift;
-          }
+          for (int r = 0; r < RW; ++r) thf[r] = rs[r].theta_f;  // may have risen last tile
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
-            const bool ps = j >= lo[r] && j < hi[r] && L[r] >= thf[r];
+            const bool ps = static_cast<uint32_t>(j - lo[r]) < static_cast<uint32_t>(span[r]) && L[r] >= thf[r];
             const uint32_t msk = __ballot_sync(0xFFFFFFFFu, ps);
             const uint32_t key = order_key(L[r]);
             const int pos = wcnt[r] + __popc(msk & lt);
             wcnt[r] += __popc(msk);
-            uint2* dst = cand_s + (r * cap + qd * wcap + min(pos, wcap - 1));
-            if (ps && pos < wcap) *dst = make_uint2(key, static_cast<uint32_t>(j));
+            if (ps && pos < wcap) seg[r][pos] = make_uint2(key, static_cast<uint32_t>(j));
             const int hidx = r * kNB + hist_index(hist_bin(key, base[r], shift[r]));
             if (ps && mode[r] == 1 && key >= base[r]) atomicAdd(&hs[hidx], 1u);
           }
@@ -891,18 +892,23 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
 #pragma unroll
               for (int r = 0; r < RW; ++r) wcnt[r] = rs[r].wcnt[qd];
             }
-          }
-          // ---- raise the threshold from the histogram: warp qd refreshes row qd
-          // every fourth tile, the warps staggered so that one refreshes per tile
-          if (qd < RW && (t & 3) == qd && rs[qd].mode == 1) {
-            RowState& st = rs[qd];
-            const Boundary B = find_boundary(hs + qd * kNB, static_cast<uint32_t>(k), lane);
-            if (B.found && lane == 0) {
-              uint64_t th = static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin) << st.shift);
-              if (th > 0xFFFFFFFFull) th = 0xFFFFFFFFull;
-              if (static_cast<uint32_t>(th) > st.theta) {
-                st.theta = static_cast<uint32_t>(th);
-                st.theta_f = theta_float(st.theta);
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {  // histogram windows may have opened
+              mode[r] = rs[r].mode;
+              base[r] = rs[r].base;
+              shift[r] = rs[r].shift;
+            }
+            // ---- raise the threshold from the histogram (warp qd for row qd)
+            if (qd < RW && mode[qd] == 1) {
+              RowState& st = rs[qd];
+              const Boundary B = find_boundary(hs + qd * kNB, static_cast<uint32_t>(k), lane);
+              if (B.found && lane == 0) {
+                uint64_t th = static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin) << st.shift);
+                if (th > 0xFFFFFFFFull) th = 0xFFFFFFFFull;
+                if (static_cast<uint32_t>(th) > st.theta) {
+                  st.theta = static_cast<uint32_t>(th);
+                  st.theta_f = theta_float(st.theta);
+                }
               }
             }
           }
