@@ -16,7 +16,7 @@
 #include "kernels.cuh"
 
 namespace fp8idx {
-__device__ int g_logits_status;  // device status of the last fp8idx_mqa_logits call
+__device__ int g_logits_status[kStatusBytes / 4];  // status block of the last fp8idx_mqa_logits call
 
 // Fixed scratch of fp8idx_mqa_logits_topk_noalloc: a module-scope device
 // array, so it is created when the library's device code is loaded on a GPU
@@ -111,7 +111,7 @@ struct Plan {
   int num_units = 0;
   int grid = 0;
   int cap = 0;
-  size_t off_cand = 0, off_scratch = 0, off_part = 0, off_cnt = 0, total = 0;
+  size_t off_cand = 0, off_scratch = 0, off_part = 0, off_cnt = 0, off_theta = 0, total = 0;
 };
 
 // Room for the candidates a row collects over `keys` keys.  With a running
@@ -144,6 +144,8 @@ void finish_plan(Plan& pl, int64_t groups, int sms, int topk, int64_t axis) {
     off += round_up(static_cast<int64_t>(pl.num_units) * pl.R * topk * 8, 256);
     pl.off_cnt = off;
     off += round_up(static_cast<int64_t>(pl.num_units) * pl.R * 4, 256);
+    pl.off_theta = off;  // per-row shared threshold
+    off += round_up(groups * pl.R * 4, 256);
   }
   pl.total = off;
 }
@@ -264,7 +266,7 @@ int fp8idx_mqa_logits(const uint8_t* q, const uint8_t* k, const float* s, const 
   int* status = nullptr;
   cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_logits_status);
   if (e != cudaSuccess) return cuda_fail(e, "status symbol");
-  e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  e = cudaMemsetAsync(status, 0, kStatusBytes, st);
   if (e != cudaSuccess) return cuda_fail(e, "status reset");
   p.status = status;
   p.wait_limit_ns = g_wait_limit_ns;
@@ -345,6 +347,9 @@ int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, c
   if (pl.n_chunks > 1) {
     p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
     p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
+    p.row_theta = reinterpret_cast<uint32_t*>(wsb + pl.off_theta);
+    e = cudaMemsetAsync(p.row_theta, 0, static_cast<size_t>(pl.num_units / pl.n_chunks) * pl.R * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
   }
   p.wait_limit_ns = g_wait_limit_ns;
   e = launch_indexer_prefill_topk(p, pl.grid, st);
@@ -430,6 +435,9 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
   if (pl.n_chunks > 1) {
     p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
     p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
+    p.row_theta = reinterpret_cast<uint32_t*>(wsb + pl.off_theta);
+    e = cudaMemsetAsync(p.row_theta, 0, static_cast<size_t>(pl.num_units / pl.n_chunks) * pl.R * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
   }
   p.wait_limit_ns = g_wait_limit_ns;
   e = launch_indexer_paged_topk(p, R, pl.grid, st);
@@ -526,6 +534,9 @@ int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const flo
   if (pl.n_chunks > 1) {
     p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
     p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
+    p.row_theta = reinterpret_cast<uint32_t*>(wsb + pl.off_theta);
+    e = cudaMemsetAsync(p.row_theta, 0, static_cast<size_t>(pl.num_units / pl.n_chunks) * pl.R * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
   }
   p.wait_limit_ns = g_wait_limit_ns;
   e = launch_indexer_prefill_topk(p, pl.grid, st);

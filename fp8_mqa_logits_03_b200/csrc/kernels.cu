@@ -96,7 +96,7 @@ __host__ __device__ constexpr SmemLayout smem_layout() {
   L.q = 0;
   L.stage = C::Q_BYTES;
   L.bar = L.stage + C::STAGES * C::TILE_BYTES;
-  L.misc = L.bar + 8 * (2 * C::STAGES + 12);
+  L.misc = L.bar + 8 * (2 * C::STAGES + 20);
   L.w = L.misc + 64;
   L.rows = L.w + R * kHeads * 4;
   L.meta = L.rows + 2 * R * static_cast<int>(sizeof(RowState));
@@ -477,8 +477,11 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
   uint64_t* drain = bars + 2 * S + 6;
   uint64_t* slot_full = bars + 2 * S + 7;
   uint64_t* slot_empty = bars + 2 * S + 9;
+  uint64_t* uq_full = bars + 2 * S + 11;   // unit queue, 4 entries
+  uint64_t* uq_empty = bars + 2 * S + 15;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SL.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL.misc + 4);
+  volatile int* uq = reinterpret_cast<volatile int*>(smem + SL.misc + 16);  // unit queue
   float* w_smem = reinterpret_cast<float*>(smem + SL.w);
   RowState* rstate = reinterpret_cast<RowState*>(smem + SL.rows);
   SlotMeta* smeta = reinterpret_cast<SlotMeta*>(smem + SL.meta);
@@ -501,6 +504,10 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       mbar_init(&tempty[a], 8);
       mbar_init(&slot_full[a], 8);
       mbar_init(&slot_empty[a], kSelWarps);
+    }
+    for (int x = 0; x < 4; ++x) {
+      mbar_init(&uq_full[x], 1);
+      mbar_init(&uq_empty[x], 9);  // the MMA thread and the eight epilogue warps
     }
     mbar_init(qfull, 1);
     mbar_init(qempty, 1);
@@ -533,8 +540,17 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         issued_phase[s] = 0;
       }
       bool ok = true;
-      for (int i = blockIdx.x; ok && i < p.num_units; i += gridDim.x) {
-        const int u = p.num_units - 1 - i;
+      // Dynamic schedule: units are claimed from a counter in the status block
+      // (largest first for the causal layouts) and announced to the MMA and
+      // epilogue warps through a four-entry queue; -1 ends the stream.
+      for (int n = 0; ok; ++n) {
+        const int qs = n & 3;
+        if (!wait_phase<true>(&uq_empty[qs], ((n >> 2) & 1) ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
+        const int idx = atomicAdd(p.status + kSchedWord, 1);
+        const int u = idx < p.num_units ? p.num_units - 1 - idx : -1;
+        uq[qs] = u;
+        mbar_arrive(&uq_full[qs]);
+        if (u < 0) break;
         const Unit U = get_unit<R, PAGED>(p, u);
         if (U.ntiles == 0) continue;
         if (!wait_phase<true>(qempty, qphase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
@@ -587,8 +603,12 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       bool ok = true;
       bool any = false;
       const uint32_t q_addr = smem_u32(q_smem);
-      for (int i = blockIdx.x; ok && i < p.num_units; i += gridDim.x) {
-        const int u = p.num_units - 1 - i;
+      for (int n = 0; ok; ++n) {
+        const int qs = n & 3;
+        if (!wait_phase<false>(&uq_full[qs], (n >> 2) & 1, abort_flag, p.status, limit)) { ok = false; break; }
+        const int u = uq[qs];
+        mbar_arrive(&uq_empty[qs]);
+        if (u < 0) break;
         const Unit U = get_unit<R, PAGED>(p, u);
         if (U.ntiles == 0) continue;
         if (!wait_phase<false>(qfull, qphase, abort_flag, p.status, limit)) { ok = false; break; }
@@ -640,10 +660,30 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
     uint32_t T = 0;
     bool aborted = false;
 
-    for (int i = blockIdx.x, it = 0; i < p.num_units; i += gridDim.x, ++it) {
-      const int u = p.num_units - 1 - i;
-      const Unit U = get_unit<R, PAGED>(p, u);
+    for (int it = 0;; ++it) {
+      const int qs = it & 3;
+      const bool got = wait_phase<false>(&uq_full[qs], (it >> 2) & 1, abort_flag, p.status, limit);
+      // every warp of the group must take the same branch below (named barriers)
+      if (bar_red_or(bar_id, 128, !got)) {
+        aborted = true;
+        break;
+      }
+      const int u = uq[qs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&uq_empty[qs]);
       const int slot = it & 1;
+      if (u < 0) {
+        // end of this CTA's units: tell the select group (unit -1 in the slot)
+        if (MODE == kModeTopK) {
+          wait_phase<true>(&slot_empty[slot], ((it >> 1) & 1) ^ 1, abort_flag, p.status, limit);
+          if (g == 0 && tid_wg == 0) smeta[slot].unit = -1;
+          named_bar_sync(bar_id, 128);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&slot_full[slot]);
+        }
+        break;
+      }
+      const Unit U = get_unit<R, PAGED>(p, u);
       RowState* rs = rstate + slot * R + g * RW;
       uint32_t* hs = hist_smem + (slot * R + g * RW) * kNB;
       uint2* cand_s = MODE == kModeTopK
@@ -898,16 +938,28 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
               base[r] = rs[r].base;
               shift[r] = rs[r].shift;
             }
-            // ---- raise the threshold from the histogram (warp qd for row qd)
-            if (qd < RW && mode[qd] == 1) {
+            // ---- raise the threshold from the histogram (warp qd for row qd).  With the
+            // key axis split over several units, the row's bound is shared through
+            // global memory: any unit's histogram bound (at least k keys of the row
+            // lie at or above it) is a bound for the whole row.
+            if (qd < RW && g * RW + qd < U.nrows) {
               RowState& st = rs[qd];
-              const Boundary B = find_boundary(hs + qd * kNB, static_cast<uint32_t>(k), lane);
-              if (B.found && lane == 0) {
-                uint64_t th = static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin) << st.shift);
-                if (th > 0xFFFFFFFFull) th = 0xFFFFFFFFull;
-                if (static_cast<uint32_t>(th) > st.theta) {
-                  st.theta = static_cast<uint32_t>(th);
-                  st.theta_f = theta_float(st.theta);
+              uint32_t th = 0;
+              if (mode[qd] == 1) {
+                const Boundary B = find_boundary(hs + qd * kNB, static_cast<uint32_t>(k), lane);
+                if (B.found) {
+                  const uint64_t t64 = static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin) << st.shift);
+                  th = t64 > 0xFFFFFFFFull ? 0xFFFFFFFFu : static_cast<uint32_t>(t64);
+                }
+              }
+              if (lane == 0) {
+                if (p.n_chunks > 1) {
+                  const uint32_t gbound = atomicMax(p.row_theta + U.row0 + g * RW + qd, th);
+                  th = max(th, gbound);
+                }
+                if (th > st.theta) {
+                  st.theta = th;
+                  st.theta_f = theta_float(th);
                 }
               }
             }
@@ -934,11 +986,12 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
     const int k = p.topk;
     const int cap = p.cand_cap;
     const int wcap = cap >> 2;
-    for (int i = blockIdx.x, it = 0; i < p.num_units; i += gridDim.x, ++it) {
+    for (int it = 0;; ++it) {
       const int slot = it & 1;
       const bool ok = wait_phase<true>(&slot_full[slot], (it >> 1) & 1, abort_flag, p.status, limit);
       if (bar_red_or(kSelBar, NT, !ok || *abort_flag)) break;
       const SlotMeta meta = smeta[slot];
+      if (meta.unit < 0) break;
       for (int rl = 0; rl < R; ++rl) {
         const RowState st = rstate[slot * R + rl];
         const uint32_t* h = hist_smem + (slot * R + rl) * kNB;

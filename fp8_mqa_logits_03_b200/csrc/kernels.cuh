@@ -26,6 +26,7 @@ constexpr int kStatCompactions = 1;     // in-stream exact compactions of a full
 constexpr int kStatGeneralSelects = 2;  // final selects that needed the general radix path
 constexpr int kStatCandidates = 3;      // candidates appended, summed over rows
 constexpr int kStatMaxBoundary = 4;     // largest boundary-bin population seen
+constexpr int kSchedWord = 16;          // status-block word: next unit for dynamic scheduling
 
 enum Mode : int { kModeLogits = 0, kModeTopK = 1 };
 
@@ -59,6 +60,7 @@ struct IndexerParams {
   uint2* scratch;   // [gridDim.x][8 epilogue warps][topk]: staging of a rare in-kernel compaction
   uint2* part;      // split mode: [num_units][R][topk]
   int* part_cnt;    // split mode: [num_units][R]
+  uint32_t* row_theta;  // split mode: [m] best lower bound on each row's k-th order key, zeroed per call
   unsigned long long wait_limit_ns;
 };
 
