@@ -992,6 +992,18 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       if (bar_red_or(kSelBar, NT, !ok || *abort_flag)) break;
       const SlotMeta meta = smeta[slot];
       if (meta.unit < 0) break;
+      // The unit's candidate segments were written one unit ago and have
+      // mostly left L2: bring every row's segments back in one go, so that
+      // the row-by-row passes below wait on L2 rather than on DRAM.
+      if (stid < R && stid < meta.nrows) {
+        const RowState& st = rstate[slot * R + stid];
+        const uint2* rowbuf = p.cand + (static_cast<size_t>(blockIdx.x * 2 + slot) * R + stid) * cap;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const int c = min(st.wcnt[s], wcap);
+          if (c > 0) l2_prefetch_bulk(rowbuf + s * wcap, static_cast<uint32_t>((c + 1) & ~1) * 8u);
+        }
+      }
       for (int rl = 0; rl < R; ++rl) {
         const RowState st = rstate[slot * R + rl];
         const uint32_t* h = hist_smem + (slot * R + rl) * kNB;
