@@ -125,7 +125,7 @@ int candidate_capacity(int topk, int64_t keys) {
   const int64_t cap = static_cast<int64_t>(1.5 * expect) + 2 * kBlockKeys;
   // Each of the row's four segments must hold its share of the k kept by a
   // compaction plus the 32 keys per tile a warp may add between two votes.
-  const int64_t floor_cap = 2 * static_cast<int64_t>(topk) + 4 * (kVoteTiles + 2) * 32;
+  const int64_t floor_cap = 2 * static_cast<int64_t>(topk) + 4 * (kMaxVoteTiles + 2) * 32;
   return static_cast<int>(round_up(std::max<int64_t>(cap, floor_cap), kBlockKeys));
 }
 

@@ -60,6 +60,7 @@ constexpr int kSelWarps = 2;     // warps in the select group
 constexpr int kSelBar = 3;       // its named barrier
 constexpr int kUpCap = kMaxTopK; // per select warp: keys above the boundary bin (fewer than topk in all)
 constexpr int kAtCap = 1024;     // per select warp: keys inside the boundary bin
+constexpr int kSelBatch = 16;    // candidate loads in flight per select thread
 
 // Per (slot, row) streaming state of the fused top-k.  A row's candidate
 // buffer holds four equal segments, one per TMEM lane quadrant (key block of
@@ -362,15 +363,15 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
       const int s = 2 * w + s2;
       const int pref = (s > 0 ? c[0] : 0) + (s > 1 ? c[1] : 0) + (s > 2 ? c[2] : 0);
       const uint2* seg = rowbuf + s * wcap;
-      for (int i0 = 0; i0 < c[s]; i0 += 8 * 32) {
-        uint2 v[8];
+      for (int i0 = 0; i0 < c[s]; i0 += kSelBatch * 32) {
+        uint2 v[kSelBatch];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
+        for (int t = 0; t < kSelBatch; ++t) {
           const int i = i0 + t * 32 + lane;
           if (i < c[s]) v[t] = seg[i];
         }
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
+        for (int t = 0; t < kSelBatch; ++t) {
           const int i = i0 + t * 32 + lane;
           if (i < c[s]) emit(pref + i, v[t].x, v[t].y);
         }
@@ -390,15 +391,15 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
       for (int s2 = 0; s2 < 2; ++s2) {
         const int s = 2 * w + s2;
         const uint2* seg = rowbuf + s * wcap;
-        for (int i0 = 0; i0 < c[s]; i0 += 8 * 32) {
-          uint2 v[8];
+        for (int i0 = 0; i0 < c[s]; i0 += kSelBatch * 32) {
+          uint2 v[kSelBatch];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
+          for (int t = 0; t < kSelBatch; ++t) {
             const int i = i0 + t * 32 + lane;
             v[t] = i < c[s] ? seg[i] : make_uint2(0u, 0u);
           }
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
+          for (int t = 0; t < kSelBatch; ++t) {
             const int i = i0 + t * 32 + lane;
             int bin = -1;
             if (i < c[s] && v[t].x >= st.base) bin = hist_bin(v[t].x, st.base, st.shift);
@@ -782,6 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         return __ldg(p.s + static_cast<int64_t>(pg) * kPageSize + (j % kPageSize));
       };
       float s_next = U.ntiles ? scale_of(key0) : 0.f;
+      int next_vote = vote_interval(0) - 1;  // the same tile sequence in every warp of the group
       for (int t = 0; t < U.ntiles; ++t, ++T) {
         const int j = key0 + t * kBlockKeys;
         const float sj = 0.5f * s_next;  // relu_dot32_x2 returns twice the head sum
@@ -832,15 +834,16 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
             const int hidx = r * kNB + hist_index(hist_bin(key, base[r], shift[r]));
             if (ps && mode[r] == 1 && key >= base[r]) atomicAdd(&hs[hidx], 1u);
           }
-          // Every kVoteTiles tiles (and the last), one barrier carries two votes:
+          // At every vote tile (and the last), one barrier carries two votes:
           // abort (weight 1: lane 0 of each warp) and maintenance (weight 5:
           // lanes 0..4 of each warp): a row still without its histogram window
-          // has candidates, or a segment is within 32 * kVoteTiles of full.
-          if ((t % kVoteTiles) == kVoteTiles - 1 || t + 1 == U.ntiles) {
+          // has candidates, or a segment is within 32 * kMaxVoteTiles of full.
+          if (t == next_vote || t + 1 == U.ntiles) {
+            next_vote = t + vote_interval(t + 1);
             bool maint = false;
 #pragma unroll
             for (int r = 0; r < RW; ++r) {
-              maint |= (mode[r] == 0 && wcnt[r] > 0) || wcnt[r] > wcap - kVoteTiles * 32;
+              maint |= (mode[r] == 0 && wcnt[r] > 0) || wcnt[r] > wcap - kMaxVoteTiles * 32;
               if (wcnt[r] > wcap && lane == 0) atomicOr(p.status, kStatusCandOverflow);
             }
             if (lane == 0) {
@@ -860,7 +863,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
               for (int r = 0; r < RW; ++r) {
                 const RowState& st = rs[r];
                 opened[r] = st.mode == 0 && (st.wcnt[0] + st.wcnt[1] + st.wcnt[2] + st.wcnt[3]) > 0;
-                compact[r] = max(max(st.wcnt[0], st.wcnt[1]), max(st.wcnt[2], st.wcnt[3])) > wcap - kVoteTiles * 32;
+                compact[r] = max(max(st.wcnt[0], st.wcnt[1]), max(st.wcnt[2], st.wcnt[3])) > wcap - kMaxVoteTiles * 32;
               }
               named_bar_sync(bar_id, 128);
               if (qd < RW && (compact[qd] || opened[qd])) {
@@ -869,7 +872,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
                 uint32_t* h = hs + qd * kNB;
                 if (opened[qd]) {
                   // Open the row's histogram window over twice the span of the keys
-                  // collected so far (at most kVoteTiles tiles' worth) and count them.
+                  // collected so far (at most kMaxVoteTiles tiles' worth) and count them.
                   uint32_t kmin = 0xFFFFFFFFu, kmax = 0;
                   for (int s = 0; s < 4; ++s)
                     for (int e = lane; e < st.wcnt[s]; e += 32) {
@@ -993,18 +996,19 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       const SlotMeta meta = smeta[slot];
       if (meta.unit < 0) break;
       // The unit's candidate segments were written one unit ago and have
-      // mostly left L2: bring every row's segments back in one go, so that
-      // the row-by-row passes below wait on L2 rather than on DRAM.
-      if (stid < R && stid < meta.nrows) {
-        const RowState& st = rstate[slot * R + stid];
-        const uint2* rowbuf = p.cand + (static_cast<size_t>(blockIdx.x * 2 + slot) * R + stid) * cap;
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const int c = min(st.wcnt[s], wcap);
-          if (c > 0) l2_prefetch_bulk(rowbuf + s * wcap, static_cast<uint32_t>((c + 1) & ~1) * 8u);
+      // mostly left L2: each row's segments are brought back two rows ahead
+      // of its pass (thread `stid` of the group prefetches segment `stid`).
+      auto prefetch_row = [&](int rl) {
+        if (stid < 4 && rl < meta.nrows) {
+          const int c = min(rstate[slot * R + rl].wcnt[stid], wcap);
+          const uint2* seg = p.cand + (static_cast<size_t>(blockIdx.x * 2 + slot) * R + rl) * cap + stid * wcap;
+          if (c > 0) l2_prefetch_bulk(seg, static_cast<uint32_t>((c + 1) & ~1) * 8u);
         }
-      }
+      };
+      prefetch_row(0);
+      prefetch_row(1);
       for (int rl = 0; rl < R; ++rl) {
+        prefetch_row(rl + 2);
         const RowState st = rstate[slot * R + rl];
         const uint32_t* h = hist_smem + (slot * R + rl) * kNB;
         const uint2* rowbuf = p.cand + (static_cast<size_t>(blockIdx.x * 2 + slot) * R + rl) * cap;
