@@ -387,6 +387,14 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
       uint2* at_w = at_all + w * kAtCap;
       uint32_t nu = 0, na = 0;  // warp-uniform counters
       const uint32_t lt = (1u << lane) - 1u;
+      // The boundary bin as a key interval [lo_key, hi_key): a key is above
+      // the bin iff key >= hi_key (never when the bin is the top, clamped one).
+      // (The bin holds at least one key, so its lower edge is below 2^32.)
+      const uint32_t lo_key = static_cast<uint32_t>(
+          min(static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin) << st.shift), static_cast<uint64_t>(0xFFFFFFFFu)));
+      const uint64_t hi64 = static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin + 1) << st.shift);
+      const bool has_hi = B.bin < kNB - 1 && hi64 <= 0xFFFFFFFFull;
+      const uint32_t hi_key = has_hi ? static_cast<uint32_t>(hi64) : 0xFFFFFFFFu;
 #pragma unroll
       for (int s2 = 0; s2 < 2; ++s2) {
         const int s = 2 * w + s2;
@@ -400,10 +408,9 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
           }
 #pragma unroll
           for (int t = 0; t < kSelBatch; ++t) {
-            const int i = i0 + t * 32 + lane;
-            int bin = -1;
-            if (i < c[s] && v[t].x >= st.base) bin = hist_bin(v[t].x, st.base, st.shift);
-            const bool up = bin > B.bin, at = bin == B.bin;
+            const bool valid = i0 + t * 32 + lane < c[s];
+            const bool up = valid && has_hi && v[t].x >= hi_key;
+            const bool at = valid && !up && v[t].x >= lo_key;
             const uint32_t mu = __ballot_sync(0xFFFFFFFFu, up);
             const uint32_t ma = __ballot_sync(0xFFFFFFFFu, at);
             if (up) {
@@ -830,9 +837,9 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
             const uint32_t key = order_key(L[r]);
             const int pos = wcnt[r] + __popc(msk & lt);
             wcnt[r] += __popc(msk);
-            if (ps && pos < wcap) seg[r][pos] = make_uint2(key, static_cast<uint32_t>(j));
+            st_global_v2_if(ps && pos < wcap, seg[r] + pos, key, static_cast<uint32_t>(j));
             const int hidx = r * kNB + hist_index(hist_bin(key, base[r], shift[r]));
-            if (ps && mode[r] == 1 && key >= base[r]) atomicAdd(&hs[hidx], 1u);
+            red_shared_add_if(ps && mode[r] == 1 && key >= base[r], hs + hidx, 1u);
           }
           // At every vote tile (and the last), one barrier carries two votes:
           // abort (weight 1: lane 0 of each warp) and maintenance (weight 5:

@@ -16,12 +16,12 @@ constexpr int kThreads = 384;      // 12 warps: TMA, MMA, 8 epilogue, 2 select
 constexpr int kStatusBytes = 256;  // device status block at the head of every workspace
 // Tiles between two group votes of the fused epilogue, after t tiles of the
 // unit: short early, where the running threshold still moves fast, and
-// growing with the tiles already streamed (clamp(t / 8, min, max)), since the
+// growing with the tiles already streamed (clamp(t / 4, min, max)), since the
 // threshold's relative movement per tile falls like 1 / t.
 constexpr int kMinVoteTiles = 4;
 constexpr int kMaxVoteTiles = 16;
 __host__ __device__ constexpr int vote_interval(int t) {
-  return t / 8 < kMinVoteTiles ? kMinVoteTiles : (t / 8 > kMaxVoteTiles ? kMaxVoteTiles : t / 8);
+  return t / 4 < kMinVoteTiles ? kMinVoteTiles : (t / 4 > kMaxVoteTiles ? kMaxVoteTiles : t / 4);
 }
 
 // device status bits (workspace word 0)

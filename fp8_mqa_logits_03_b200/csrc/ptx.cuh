@@ -102,6 +102,22 @@ __device__ __forceinline__ void l2_prefetch_bulk(const void* src, uint32_t bytes
                : "memory");
 }
 
+// Predicated stores and reductions: one instruction under a predicate, so
+// that a per-lane condition costs no branch.  No memory clobber: callers
+// order them against later readers with a barrier.
+__device__ __forceinline__ void st_global_v2_if(bool pred, void* p, uint32_t a, uint32_t b) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t@q st.global.v2.u32 [%1], {%2, %3};\n\t}" ::"r"(
+          static_cast<uint32_t>(pred)),
+      "l"(reinterpret_cast<uint64_t>(p)), "r"(a), "r"(b));
+}
+__device__ __forceinline__ void red_shared_add_if(bool pred, uint32_t* p, uint32_t v) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t@q red.shared.add.u32 [%1], %2;\n\t}" ::"r"(
+          static_cast<uint32_t>(pred)),
+      "r"(smem_u32(p)), "r"(v));
+}
+
 // ---------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
