@@ -347,20 +347,21 @@ struct TwoListSrc {
 
 // Exact top-k of one finished row by the select group (two warps; warp w
 // reads segments 2w and 2w+1).  emit(pos, key, index) receives positions
-// [0, returned count).  Keys above the histogram's boundary bin are in; the
-// boundary bin is resolved exactly in shared memory; anything unusual falls
-// back to a radix select over the whole buffer.
-template <class Emit>
+// [0, returned count).  FAST (G = 1 or 2 warps, G * (kUpCap + kAtCap)
+// staging pairs in up_all / at_all): keys above the histogram's boundary bin
+// are in and the boundary bin is resolved exactly in shared memory; anything
+// unusual, and every row when !FAST, takes a radix select over the whole buffer.
+template <bool FAST, int G, class Emit>
 __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& st, const uint32_t* h,
-                                int k, const Group<kSelWarps>& g, uint2* up_all, uint2* at_all,
+                                int k, const Group<G>& g, uint2* up_all, uint2* at_all,
                                 uint32_t* xchg, int* stats, Emit emit) {
+  static_assert(!FAST || G <= 2, "the staged path exchanges counts between at most two warps");
   const int w = g.warp(), lane = g.lane();
   const int c[4] = {st.wcnt[0], st.wcnt[1], st.wcnt[2], st.wcnt[3]};
   const int cnt = c[0] + c[1] + c[2] + c[3];
   if (cnt <= k) {
 #pragma unroll
-    for (int s2 = 0; s2 < 2; ++s2) {
-      const int s = 2 * w + s2;
+    for (int s = w; s < 4; s += G) {
       const int pref = (s > 0 ? c[0] : 0) + (s > 1 ? c[1] : 0) + (s > 2 ? c[2] : 0);
       const uint2* seg = rowbuf + s * wcap;
       for (int i0 = 0; i0 < c[s]; i0 += kSelBatch * 32) {
@@ -379,7 +380,7 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
     }
     return cnt;
   }
-  if (st.mode == 1) {
+  if (FAST && st.mode == 1) {
     const Boundary B = find_boundary(h, static_cast<uint32_t>(k), lane);
     if (B.found) {
       if (g.tid == 0) atomicMax(reinterpret_cast<unsigned*>(stats + kStatMaxBoundary), B.inbin);
@@ -396,8 +397,7 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
       const bool has_hi = B.bin < kNB - 1 && hi64 <= 0xFFFFFFFFull;
       const uint32_t hi_key = has_hi ? static_cast<uint32_t>(hi64) : 0xFFFFFFFFu;
 #pragma unroll
-      for (int s2 = 0; s2 < 2; ++s2) {
-        const int s = 2 * w + s2;
+      for (int s = w; s < 4; s += G) {
         const uint2* seg = rowbuf + s * wcap;
         for (int i0 = 0; i0 < c[s]; i0 += kSelBatch * 32) {
           uint2 v[kSelBatch];
@@ -426,12 +426,18 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
           }
         }
       }
-      if (lane == 0) {
-        xchg[2 * w] = nu;
-        xchg[2 * w + 1] = na;
+      uint32_t nu0 = nu, na0 = na, nu1 = 0, na1 = 0;
+      if (G > 1) {
+        if (lane == 0) {
+          xchg[2 * w] = nu;
+          xchg[2 * w + 1] = na;
+        }
+        g.sync();
+        nu0 = xchg[0];
+        na0 = xchg[1];
+        nu1 = xchg[2];
+        na1 = xchg[3];
       }
-      g.sync();
-      const uint32_t nu0 = xchg[0], na0 = xchg[1], nu1 = xchg[2], na1 = xchg[3];
       const bool consistent = nu0 + nu1 == B.above && na0 + na1 == B.inbin &&
                               nu0 <= static_cast<uint32_t>(kUpCap) && nu1 <= static_cast<uint32_t>(kUpCap) &&
                               na0 <= static_cast<uint32_t>(kAtCap) && na1 <= static_cast<uint32_t>(kAtCap);
@@ -442,8 +448,8 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
         const int need = k - static_cast<int>(B.above);
         const TwoListSrc src{at_all, static_cast<int>(na0), at_all + kAtCap, static_cast<int>(na1)};
         const int tot = static_cast<int>(na0 + na1);
-        const SelectResult sel = group_select<kSelWarps>(src, tot, need, g);
-        const int n2 = group_emit<kSelWarps>(src, tot, sel, g, [&](int pos, uint64_t K) {
+        const SelectResult sel = group_select<G>(src, tot, need, g);
+        const int n2 = group_emit<G>(src, tot, sel, g, [&](int pos, uint64_t K) {
           emit(static_cast<int>(B.above) + pos, composite_value(K), composite_index(K));
         });
         return static_cast<int>(B.above) + n2;
@@ -451,12 +457,48 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
     }
   }
   // general path: radix select over the whole buffer
-  if (g.tid == 0) atomicAdd(stats + kStatGeneralSelects, 1);
+  if (FAST && g.tid == 0) atomicAdd(stats + kStatGeneralSelects, 1);
   const SegSrc src{rowbuf, wcap, c[0], c[1], c[2], c[3]};
-  const SelectResult sel = group_select<kSelWarps>(src, 4 * wcap, k, g);
-  return group_emit<kSelWarps>(src, 4 * wcap, sel, g, [&](int pos, uint64_t K) {
+  const SelectResult sel = group_select<G>(src, 4 * wcap, k, g);
+  return group_emit<G>(src, 4 * wcap, sel, g, [&](int pos, uint64_t K) {
     emit(pos, composite_value(K), composite_index(K));
   });
+}
+
+// Exact top-k of one finished row (row rl of a slot) written out: the final
+// list (-1 / -inf padded) with one key chunk, else the unit's partial list and
+// its length.
+template <bool FAST, int R, int G>
+__device__ void write_row_topk(const IndexerParams& p, const SlotMeta& meta, int rl, const RowState& st,
+                               const uint32_t* h, const uint2* rowbuf, const Group<G>& g,
+                               uint2* up_all, uint2* at_all, uint32_t* xchg) {
+  const int k = p.topk;
+  const int wcap = p.cand_cap >> 2;
+  const bool present = rl < meta.nrows;
+  const int cnt = st.wcnt[0] + st.wcnt[1] + st.wcnt[2] + st.wcnt[3];
+  if (present && g.tid == 0) atomicAdd(p.status + kStatCandidates, cnt);
+  if (p.n_chunks == 1) {
+    if (!present) return;
+    const int row = meta.row0 + rl;
+    int32_t* orow = p.out_idx + static_cast<int64_t>(row) * k;
+    float* vrow = p.out_vals ? p.out_vals + static_cast<int64_t>(row) * k : nullptr;
+    const int nout = final_select_row<FAST>(rowbuf, wcap, st, h, k, g, up_all, at_all, xchg, p.status,
+                                            [&](int pos, uint32_t key, uint32_t j) {
+                                              orow[pos] = static_cast<int32_t>(j);
+                                              if (vrow) vrow[pos] = key_to_float(key);
+                                            });
+    for (int pos = nout + g.tid; pos < k; pos += 32 * G) {
+      orow[pos] = -1;
+      if (vrow) vrow[pos] = -INFINITY;
+    }
+  } else {
+    uint2* prow = p.part + (static_cast<size_t>(meta.unit) * R + rl) * k;
+    int nout = 0;
+    if (present && cnt > 0)
+      nout = final_select_row<FAST>(rowbuf, wcap, st, h, k, g, up_all, at_all, xchg, p.status,
+                                    [&](int pos, uint32_t key, uint32_t j) { prow[pos] = make_uint2(key, j); });
+    if (g.tid == 0) p.part_cnt[static_cast<size_t>(meta.unit) * R + rl] = nout;
+  }
 }
 
 // ------------------------------------------------------------------ kernel
@@ -468,6 +510,8 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
   constexpr int N = C::N;
   constexpr int RW = C::RW;
   constexpr int S = C::STAGES;
+  static_assert(4 * (kUpCap + kAtCap) * 8 <= SL.stage + S * C::TILE_BYTES,
+                "end-of-kernel select staging must fit in the q and key-tile buffers");
 
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base (128-byte swizzled TMA tiles), derived by pointer
@@ -490,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SL.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL.misc + 4);
   volatile int* uq = reinterpret_cast<volatile int*>(smem + SL.misc + 16);  // unit queue
+  int* claim = reinterpret_cast<int*>(smem + SL.misc + 32);  // rows of each slot handed out so far
   float* w_smem = reinterpret_cast<float*>(smem + SL.w);
   RowState* rstate = reinterpret_cast<RowState*>(smem + SL.rows);
   SlotMeta* smeta = reinterpret_cast<SlotMeta*>(smem + SL.meta);
@@ -681,8 +726,32 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       if (lane == 0) mbar_arrive(&uq_empty[qs]);
       const int slot = it & 1;
       if (u < 0) {
-        // end of this CTA's units: tell the select group (unit -1 in the slot)
         if (MODE == kModeTopK) {
+          // Out of units.  Warpgroup 0 takes rows of the last two units off
+          // the select group, which may still be busy with them: each warp
+          // claims a row and selects it alone, staging in the q and key-tile
+          // buffers (every MMA of this CTA has completed, so they are free).
+          // The CTA then does not finish on the select group's two warps.
+          if (g == 0) {
+            uint2* up_h = reinterpret_cast<uint2*>(smem) + qd * (kUpCap + kAtCap);
+            for (int back = 2; back >= 1; --back) {
+              if (it < back) continue;
+              const int hslot = (it - back) & 1;
+              if (!wait_phase<true>(&slot_full[hslot], ((it - back) >> 1) & 1, abort_flag, p.status, limit)) break;
+              const SlotMeta meta = smeta[hslot];
+              for (;;) {
+                int rl = 0;
+                if (lane == 0) rl = atomicAdd(claim + hslot, 1);
+                rl = __shfl_sync(0xFFFFFFFFu, rl, 0);
+                if (rl >= R) break;
+                write_row_topk<true, R>(p, meta, rl, rstate[hslot * R + rl], hist_smem + (hslot * R + rl) * kNB,
+                                        p.cand + (static_cast<size_t>(blockIdx.x * 2 + hslot) * R + rl) * cap, grp,
+                                        up_h, up_h + kUpCap, nullptr);
+                __syncwarp();
+              }
+            }
+          }
+          // tell the select group (unit -1 in the slot)
           wait_phase<true>(&slot_empty[slot], ((it >> 1) & 1) ^ 1, abort_flag, p.status, limit);
           if (g == 0 && tid_wg == 0) smeta[slot].unit = -1;
           named_bar_sync(bar_id, 128);
@@ -739,6 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         }
         for (int x = tid_wg; x < RW * kNB; x += 128) hs[x] = 0;
         if (g == 0 && tid_wg == 0) {
+          claim[slot] = 0;
           smeta[slot].unit = u;
           smeta[slot].row0 = U.row0;
           smeta[slot].nrows = U.nrows;
@@ -993,7 +1063,6 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
     constexpr int NT = 32 * kSelWarps;
     Group<kSelWarps> grp{ssel_smem, ssel_smem + 256, ssel_smem + 300, kSelBar, stid};
     uint32_t* xchg = ssel_smem + 304;
-    const int k = p.topk;
     const int cap = p.cand_cap;
     const int wcap = cap >> 2;
     for (int it = 0;; ++it) {
@@ -1014,36 +1083,18 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       };
       prefetch_row(0);
       prefetch_row(1);
-      for (int rl = 0; rl < R; ++rl) {
+      // Rows are claimed one at a time from the slot's counter: the epilogue
+      // warps, once out of units, claim the last unit's remaining rows too.
+      for (;;) {
+        if (stid == 0) xchg[8] = static_cast<uint32_t>(atomicAdd(claim + slot, 1));
+        grp.sync();
+        const int rl = static_cast<int>(xchg[8]);
+        if (rl >= R) break;
         prefetch_row(rl + 2);
         const RowState st = rstate[slot * R + rl];
-        const uint32_t* h = hist_smem + (slot * R + rl) * kNB;
-        const uint2* rowbuf = p.cand + (static_cast<size_t>(blockIdx.x * 2 + slot) * R + rl) * cap;
-        const bool present = rl < meta.nrows;
-        const int cnt = st.wcnt[0] + st.wcnt[1] + st.wcnt[2] + st.wcnt[3];
-        if (present && stid == 0) atomicAdd(p.status + kStatCandidates, cnt);
-        if (p.n_chunks == 1) {
-          if (!present) continue;
-          const int row = meta.row0 + rl;
-          int32_t* orow = p.out_idx + static_cast<int64_t>(row) * k;
-          float* vrow = p.out_vals ? p.out_vals + static_cast<int64_t>(row) * k : nullptr;
-          const int nout = final_select_row(rowbuf, wcap, st, h, k, grp, up_smem, at_smem, xchg, p.status,
-                                            [&](int pos, uint32_t key, uint32_t j) {
-                                              orow[pos] = static_cast<int32_t>(j);
-                                              if (vrow) vrow[pos] = key_to_float(key);
-                                            });
-          for (int pos = nout + stid; pos < k; pos += NT) {
-            orow[pos] = -1;
-            if (vrow) vrow[pos] = -INFINITY;
-          }
-        } else {
-          uint2* prow = p.part + (static_cast<size_t>(meta.unit) * R + rl) * k;
-          int nout = 0;
-          if (present && cnt > 0)
-            nout = final_select_row(rowbuf, wcap, st, h, k, grp, up_smem, at_smem, xchg, p.status,
-                                    [&](int pos, uint32_t key, uint32_t j) { prow[pos] = make_uint2(key, j); });
-          if (stid == 0) p.part_cnt[static_cast<size_t>(meta.unit) * R + rl] = nout;
-        }
+        write_row_topk<true, R>(p, meta, rl, st, hist_smem + (slot * R + rl) * kNB,
+                                p.cand + (static_cast<size_t>(blockIdx.x * 2 + slot) * R + rl) * cap, grp,
+                                up_smem, at_smem, xchg);
         grp.sync();
       }
       __syncwarp();
