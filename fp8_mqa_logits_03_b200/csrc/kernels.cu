@@ -1129,27 +1129,81 @@ struct PartSrc {
   }
 };
 
-constexpr int kMergeWarps = 8;
+// A row's partial lists gathered densely in shared memory.
+struct DenseSrc {
+  const uint2* a;
+  __device__ __forceinline__ bool get(int e, uint64_t& K) const {
+    const uint2 v = a[e];
+    K = compose_key(v.x, v.y);
+    return true;
+  }
+};
 
+constexpr int kMergeWarps = 8;
+constexpr int kMergeMaxChunks = kMergeWarps * 32;  // one chunk count per thread
+constexpr int kMergeStage = 24576;                 // pairs a row can gather in shared memory (192 KB)
+
+// One CTA per row.  The chunk counts are scanned into offsets; when the
+// row's surviving pairs fit, they are gathered densely into shared memory and
+// selected there, else the select reads the partial lists in place.
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergeParams p) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t red[8 * kMergeWarps];
   __shared__ uint32_t counter;
+  __shared__ int pre[kMergeMaxChunks + 1];
+  __shared__ int wsum[kMergeWarps];
+  extern __shared__ uint2 stage[];  // kMergeStage pairs (dynamic)
   const int row = blockIdx.x;
   const int unit_row = row / p.R;  // row block / request
   const int rl = row - unit_row * p.R;
   const size_t u0 = static_cast<size_t>(unit_row) * p.n_chunks;
-  PartSrc src{p.part + (u0 * p.R + rl) * p.topk, p.part_cnt + u0 * p.R + rl,
-              static_cast<size_t>(p.R) * p.topk, p.R, p.topk};
+  const uint2* base = p.part + (u0 * p.R + rl) * p.topk;
+  const size_t stride = static_cast<size_t>(p.R) * p.topk;
+  const int* cnt = p.part_cnt + u0 * p.R + rl;
   Group<kMergeWarps> g{hist, red, &counter, 1, static_cast<int>(threadIdx.x)};
-  const int total = p.n_chunks * p.topk;
-  const SelectResult sel = group_select<kMergeWarps>(src, total, p.topk, g);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int total = -1;  // pairs surviving in all chunks (-1: not scanned)
+  if (p.n_chunks <= kMergeMaxChunks) {
+    const int c = threadIdx.x;
+    const int v = c < p.n_chunks ? __ldg(cnt + static_cast<size_t>(c) * p.R) : 0;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += t;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    if (c < p.n_chunks) pre[c] = before + incl - v;
+    if (c == kMergeMaxChunks - 1) pre[p.n_chunks] = before + incl;
+    __syncthreads();
+    total = pre[p.n_chunks];
+  }
   int32_t* orow = p.out_idx + static_cast<int64_t>(row) * p.topk;
   float* vrow = p.out_vals ? p.out_vals + static_cast<int64_t>(row) * p.topk : nullptr;
-  const int nout = group_emit<kMergeWarps>(src, total, sel, g, [&](int pos, uint64_t K) {
+  auto emit = [&](int pos, uint64_t K) {
     orow[pos] = static_cast<int32_t>(composite_index(K));
     if (vrow) vrow[pos] = key_to_float(composite_value(K));
-  });
+  };
+  int nout;
+  if (total >= 0 && total <= kMergeStage) {
+    for (int c = warp; c < p.n_chunks; c += kMergeWarps) {
+      const uint2* src = base + static_cast<size_t>(c) * stride;
+      const int n = pre[c + 1] - pre[c];
+      for (int i = lane; i < n; i += 32) stage[pre[c] + i] = src[i];
+    }
+    __syncthreads();
+    const DenseSrc src{stage};
+    const SelectResult sel = group_select<kMergeWarps>(src, total, p.topk, g);
+    nout = group_emit<kMergeWarps>(src, total, sel, g, emit);
+  } else {
+    const PartSrc src{base, cnt, stride, p.R, p.topk};
+    const int all = p.n_chunks * p.topk;
+    const SelectResult sel = group_select<kMergeWarps>(src, all, p.topk, g);
+    nout = group_emit<kMergeWarps>(src, all, sel, g, emit);
+  }
   for (int pos = nout + threadIdx.x; pos < p.topk; pos += blockDim.x) {
     orow[pos] = -1;
     if (vrow) vrow[pos] = -INFINITY;
@@ -1221,7 +1275,10 @@ cudaError_t launch_indexer_paged_topk(const IndexerParams& p, int R, int grid, c
 }
 
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t st) {
-  merge_kernel<<<p.rows, kMergeWarps * 32, 0, st>>>(p);
+  constexpr int smem = kMergeStage * static_cast<int>(sizeof(uint2));
+  cudaError_t e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  merge_kernel<<<p.rows, kMergeWarps * 32, smem, st>>>(p);
   return cudaGetLastError();
 }
 
