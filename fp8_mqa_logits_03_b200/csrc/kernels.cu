@@ -594,13 +594,23 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       }
       bool ok = true;
       // Dynamic schedule: units are claimed from a counter in the status block
-      // (largest first for the causal layouts) and announced to the MMA and
-      // epilogue warps through a four-entry queue; -1 ends the stream.
+      // and announced to the MMA and epilogue warps through a four-entry
+      // queue; -1 ends the stream.  Whole-row units go last row block first
+      // (the largest, in the causal layouts).  With a split key axis the order
+      // is chunk-major: every row block's (request's) first chunk, then every
+      // second one, and so on, so that full chunks come before the short last
+      // ones and a row's later chunks start from the threshold its earlier
+      // chunks raised.
       for (int n = 0; ok; ++n) {
         const int qs = n & 3;
         if (!wait_phase<true>(&uq_empty[qs], ((n >> 2) & 1) ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
         const int idx = atomicAdd(p.status + kSchedWord, 1);
-        const int u = idx < p.num_units ? p.num_units - 1 - idx : -1;
+        int u = -1;
+        if (idx < p.num_units) {
+          const int groups = p.num_units / p.n_chunks;
+          u = p.n_chunks == 1 ? p.num_units - 1 - idx
+                              : (groups - 1 - idx % groups) * p.n_chunks + idx / groups;
+        }
         uq[qs] = u;
         mbar_arrive(&uq_full[qs]);
         if (u < 0) break;
