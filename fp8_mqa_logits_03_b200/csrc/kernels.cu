@@ -26,10 +26,13 @@
 //               state (double buffered, so it overlaps the next unit) and
 //               selects each row's exact top-k: keys above the boundary bin
 //               go straight out, the boundary bin is resolved in shared memory.
+//               Rows are claimed from a per-slot counter; once out of units,
+//               the first epilogue warpgroup claims the last units' rows too.
 // A unit is R query rows (a row block, or one request's rows in the paged
-// form) times one chunk of keys.  With one chunk per unit the fused kernel
-// writes the final top-k; with several, each unit writes its exact partial
-// top-k and the merge kernel selects from the union.
+// form) times one chunk of keys, claimed from a device counter by the
+// producer and passed on through a shared-memory queue.  With one chunk per
+// unit the fused kernel writes the final top-k; with several, each unit
+// writes its exact partial top-k and the merge kernel selects from the union.
 #include <cfloat>
 #include <climits>
 #include <cstdint>
