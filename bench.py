@@ -16,6 +16,11 @@ memory and the top-k indices copied back inside each timed step.
 
 --impl reference times the float64 CPU oracle instead, on a bounded sample
 of the same workload's rows per step (rank 0 only).
+
+--path chained times the unfused comparison path instead: materialised
+logits (fp8idx_mqa_logits, rows chunked so that one chunk of logits stays
+within 2 GiB) followed by fp8idx_topk_rows on each chunk, the loop of the
+pages' chunked benchmark.  Same metric, same algorithmic flops.
 """
 from __future__ import annotations
 
@@ -49,11 +54,15 @@ def strict_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, choices=sorted(workloads.WORKLOADS), default=WORKLOAD,
                     help="workload index (default 1, the headline causal prefill)")
+    ap.add_argument("--path", choices=["fused", "chained"], default="fused",
+                    help="fused logits + top-k (default) or materialised logits then top-k")
     ap.add_argument("--quick", action="store_true",
                     help="device timing only: skip the end-to-end pass and the CPU baseline")
     a = ap.parse_args(argv)
     if a.gpus < 1 or a.steps < 1 or a.warmup < 3:
         ap.error("need --gpus >= 1, --steps >= 1, --warmup >= 3")
+    if a.path == "chained" and (a.workload == 4 or a.impl == "reference"):
+        ap.error("--path chained is the prefill comparison path of our implementation")
     return a
 
 
@@ -246,7 +255,10 @@ def cpu_baseline(d, budget_s: float = 12.0):
 
 # ----------------------------------------------------------------------------- our arm
 
-def make_case(fx, index, dev):
+CHUNK_BYTES = 2 << 30  # logits bytes per row chunk of the chained path
+
+
+def make_case(fx, index, dev, path="fused"):
     """Device-resident inputs, outputs, workspace and the C-ABI call for one workload."""
     d = workloads.make_workload(index)
     topk = workloads.TOPK
@@ -283,9 +295,28 @@ def make_case(fx, index, dev):
             fx.mqa_logits_topk(**dv, topk=topk, out=out, workspace=ws)
         kernel = "indexer_kernel<8,false,1> (fused logits + top-k)"
         bound = "tensor"
+        if path == "chained":
+            m, n = d["m"], d["n"]
+            rows = max(1, min(m, CHUNK_BYTES // (4 * max(n, 1))))
+            logits = torch.empty((rows, n), dtype=torch.float32, device=dev)
+            chunks = [(r0, min(m, r0 + rows)) for r0 in range(0, m, rows)]
+
+            def call():
+                for r0, r1 in chunks:
+                    lg = logits[: r1 - r0]
+                    fx.mqa_logits(dv["q"][r0:r1], dv["k"], dv["s"], dv["w"][r0:r1], dv["ks"][r0:r1],
+                                  dv["ke"][r0:r1], logits=lg)
+                    fx.topk_rows(lg, dv["ks"][r0:r1], dv["ke"][r0:r1], topk, out=out[r0:r1])
+            kernel = (f"indexer_kernel<8,false,0> (materialised logits) + topk_rows_kernel, "
+                      f"{len(chunks)} row chunk(s) of <= {rows} rows")
+            ws = None
+            launches = 2 * len(chunks)
     out_host = torch.empty(out.shape, dtype=torch.int32).pin_memory()
+    if path == "fused":
+        launches = 2 if index in (0, 4) else 1  # + the merge kernel when the key axis is split
     return dict(d=d, call=call, host=host, dv=dv, out=out, out_host=out_host, ws=ws, pairs=pairs,
-                flops=FLOP_PER_PAIR * pairs, bytes=nbytes, kernel=kernel, bound=bound)
+                flops=FLOP_PER_PAIR * pairs, bytes=nbytes, kernel=kernel, bound=bound,
+                launches=launches)
 
 
 def run_ours(args, rank, world, local, pg):
@@ -296,7 +327,7 @@ def run_ours(args, rank, world, local, pg):
     barrier(pg)
     fx.lib()
     dev = torch.device("cuda", local)
-    case = make_case(fx, args.workload, dev)  # every rank: one independent slice of this shape
+    case = make_case(fx, args.workload, dev, args.path)  # every rank: one independent slice
     d, call, host, dv, out, out_host, ws = (case[x] for x in
                                             ("d", "call", "host", "dv", "out", "out_host", "ws"))
     pairs, flops = case["pairs"], case["flops"]
@@ -306,7 +337,7 @@ def run_ours(args, rank, world, local, pg):
     for _ in range(args.warmup):
         call()
     torch.cuda.synchronize(dev)
-    assert fx.read_device_status(ws) == 0, "device status set during warm-up"
+    assert fx.read_device_status(ws) == 0, "device status set during warm-up"  # ws None: logits call
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -325,7 +356,7 @@ def run_ours(args, rank, world, local, pg):
     ms_per_step = total_ms / args.steps
     value = world * flops * args.steps / (total_ms / 1e3) / 1e12
     status = fx.read_device_status(ws)
-    kstats = fx.read_device_stats(ws)  # counters of the last timed call
+    kstats = fx.read_device_stats(ws) if ws is not None else None  # counters of the last timed call
 
     # end to end through the same call: pinned H2D of the inputs, D2H of the top-k
     h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -379,7 +410,7 @@ def run_ours(args, rank, world, local, pg):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": None if e2e_ms is None else e2e_ms / args.steps},
-        "gpu_launches": args.steps * (2 if args.workload in (0, 4) else 1),
+        "gpu_launches": args.steps * case["launches"],
         "clocks": clocks.summary(),
         "device_status": status,
         "kernel_stats": kstats,
@@ -388,7 +419,9 @@ def run_ours(args, rank, world, local, pg):
     for key in ("m", "n", "B", "R"):
         if key in d:
             line["config"][key] = d[key]
-    if args.workload != 4 and not args.quick:
+    if args.path != "fused":
+        line["config"]["path"] = args.path
+    if args.workload != 4 and not args.quick and args.path == "fused":
         line["cpu_baseline"] = cpu_baseline(d)
     return line
 
