@@ -115,6 +115,7 @@ def _check_fused(d, idx, vals, rows, k):
     (16, 4096, 2048, 2),     # the tiny workload's shape
     (13, 9000, 2048, 3),     # split schedule, rows longer than k
     (9, 6000, 64, 4),        # small k: many in-kernel compactions
+    (11, 7000, 512, 5),      # top-512, the GLM-5.3-Flash indexer width
 ])
 def test_fused_small(m, n, k, seed):
     ks, ke = _ragged(m, n, seed)
@@ -182,7 +183,7 @@ def _paged_check(d, idx, vals, rows, k):
         check_topk_row(idx[row], ref[r], lo, hi, k, None if vals is None else vals[row], f"row {row}")
 
 
-@pytest.mark.parametrize("R,k", [(4, 2048), (8, 2048), (4, 100)])
+@pytest.mark.parametrize("R,k", [(4, 2048), (8, 2048), (4, 100), (8, 512)])
 def test_paged_small(R, k):
     lengths = [1, 3, 64, 65, 127, 128, 129, 700, 2100, 5000, 4097]
     d = workloads.make_paged(len(lengths), R, 1, 5000, seed=R + k, lengths=lengths)
