@@ -116,6 +116,8 @@ def _check_fused(d, idx, vals, rows, k):
     (13, 9000, 2048, 3),     # split schedule, rows longer than k
     (9, 6000, 64, 4),        # small k: many in-kernel compactions
     (11, 7000, 512, 5),      # top-512, the GLM-5.3-Flash indexer width
+    (10, 3000, 1, 6),        # k = 1: an argmax per row (lowest index on ties)
+    (10, 5000, 2047, 7),     # k just below the maximum, odd
 ])
 def test_fused_small(m, n, k, seed):
     ks, ke = _ragged(m, n, seed)
