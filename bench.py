@@ -337,7 +337,9 @@ def run_ours(args, rank, world, local, pg):
     for _ in range(args.warmup):
         call()
     torch.cuda.synchronize(dev)
-    assert fx.read_device_status(ws) == 0, "device status set during warm-up"  # ws None: logits call
+    warm_status = fx.read_device_status(ws)  # ws None: the last logits call's status
+    if warm_status != 0:
+        raise RuntimeError(f"device status {warm_status:#x} set during warm-up")
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
