@@ -63,6 +63,8 @@ def _load():
                                                      ctypes.c_int64, vp, ctypes.c_int]
             lib.oracle_paged_topk_rows.argtypes = [vp, ctypes.c_int64, vp, ctypes.c_int, vp,
                                                    ctypes.c_int64, ctypes.c_int, vp, vp]
+            lib.oracle_act_quant_store.argtypes = [vp, ctypes.c_int64, ctypes.c_int, vp,
+                                                   ctypes.c_int64, vp, vp]
             _lib = lib
     return _lib
 
@@ -204,3 +206,31 @@ def paged_logits_topk_rows(q, k_pages, s_pages, w, block_table, seq_lens, R: int
     lg = paged_logits_rows(q, k_pages, s_pages, w, block_table, seq_lens, R, rows, None, threads)
     idx, vals = paged_topk_rows(lg, seq_lens, R, topk, rows)
     return idx, vals, lg
+
+
+# ----------------------------------------------------------------------------
+# key quantisation into the paged pool
+# ----------------------------------------------------------------------------
+
+def act_quant_store(x_bf16, slot, num_slots: int, k_pool=None, s_pool=None):
+    """Quantise bf16 key rows to e4m3 with one fp32 scale per token and store
+    them in a pool of `num_slots` 128-byte slots (64 per page).
+
+    x_bf16: [T, D] uint16 (bf16 bit patterns); slot: [T] int64, a slot outside
+    [0, num_slots) is skipped.  k_pool [num_slots, D] uint8 and s_pool
+    [num_slots] f32 are updated in place (created zero-filled when None) and
+    returned.  s_t = max(max_d |x_t|, 1e-4) / 448 and codes = e4m3(x / s_t),
+    both in fp32.
+    """
+    lib = _load()
+    x = _c(x_bf16, np.uint16)
+    slot = _c(slot, np.int64)
+    T, D = x.shape
+    if k_pool is None:
+        k_pool = np.zeros((num_slots, D), np.uint8)
+    if s_pool is None:
+        s_pool = np.zeros((num_slots,), np.float32)
+    assert k_pool.flags.c_contiguous and k_pool.dtype == np.uint8 and k_pool.shape == (num_slots, D)
+    assert s_pool.flags.c_contiguous and s_pool.dtype == np.float32 and s_pool.shape == (num_slots,)
+    lib.oracle_act_quant_store(_p(x), T, D, _p(slot), num_slots, _p(k_pool), _p(s_pool))
+    return k_pool, s_pool

@@ -333,3 +333,46 @@ void oracle_paged_topk_rows(const double* logits, int64_t lmax, const int32_t* s
     topk_one_row(logits + r * lmax, 0, ke, k, out_idx + r * k, out_val ? out_val + r * k : NULL);
   }
 }
+
+/* ------------------------------------------------------------------ */
+/* Key quantisation into the paged key pool                           */
+/* ------------------------------------------------------------------ */
+
+/* The producer side of the paged keys: the `act_quant` step and the fp8
+ * k-pool stores that the "Serve GLM-5.3-Flash on SM80" page names (commit
+ * notes: the k-pool write kernels, stored through an e4m3fn codec).  The
+ * pages do not print the scale rule; the reading taken is one fp32 scale per
+ * token,
+ *     s_t = max(amax_t, 1e-4) / 448,   amax_t = max_d |x[t,d]|,
+ * and codes e4m3(x[t,d] / s_t) rounded to nearest even and saturated.  The
+ * scale and the quotient decide integer codes, so they are taken in fp32,
+ * the precision the library computes them in; the rounding of the fp32
+ * quotient to e4m3 is the codec above.  Token t is written to pool slot
+ * slot[t] (page slot[t] / 64, row slot[t] % 64); a slot outside
+ * [0, num_slots) means "do not store" and leaves the pool untouched. */
+static float bf16_to_float(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+void oracle_act_quant_store(const uint16_t* x, int64_t T, int D, const int64_t* slot,
+                            int64_t num_slots, uint8_t* k_pool, float* s_pool) {
+  for (int64_t t = 0; t < T; ++t) {
+    const int64_t sl = slot[t];
+    if (sl < 0 || sl >= num_slots) continue;
+    const uint16_t* row = x + t * D;
+    float amax = 0.0f;
+    for (int d = 0; d < D; ++d) {
+      const float a = fabsf(bf16_to_float(row[d]));
+      if (a > amax) amax = a;
+    }
+    const float sc = (amax > 1e-4f ? amax : 1e-4f) / 448.0f;
+    for (int d = 0; d < D; ++d) {
+      const float v = bf16_to_float(row[d]) / sc;
+      k_pool[sl * D + d] = oracle_e4m3_encode((double)v);
+    }
+    s_pool[sl] = sc;
+  }
+}

@@ -295,3 +295,69 @@ def test_workload_shapes():
     used = bt[bt >= 0]
     assert used.numel() == d["P"] and torch.unique(used).numel() == d["P"]
     assert int(d["seq_lens"].min()) >= 4096 and int(d["seq_lens"].max()) <= 8192
+
+
+# ---------------------------------------------------------------------------- key quantisation
+
+def _bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.to(torch.bfloat16).contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def test_act_quant_unit_scale_row_is_the_codec():
+    # amax exactly 448 gives the scale 1, so the codes are the codec itself
+    g = torch.Generator().manual_seed(5)
+    row = (torch.rand(128, generator=g) * 800 - 400)
+    row[17] = -448.0
+    x = _bf16_bits(row[None])
+    kp, sp = oracle.act_quant_store(x, np.array([0]), 1)
+    assert sp[0] == np.float32(1.0)
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).float().numpy()[0]
+    assert np.array_equal(kp[0], oracle.e4m3_encode(xf.astype(np.float64)))
+    assert kp[0, 17] == 0xFE  # -448
+
+
+def test_act_quant_zero_row_uses_the_floor():
+    kp, sp = oracle.act_quant_store(np.zeros((1, 128), np.uint16), np.array([0]), 1)
+    assert sp[0] == np.float32(np.float32(1e-4) / np.float32(448.0))
+    assert not kp.any()
+
+
+def test_act_quant_matches_torch_fp32_and_its_e4m3_cast():
+    # the same rule written with torch ops: fp32 amax, scale and quotient,
+    # then torch's own float -> float8_e4m3fn cast (round to nearest even)
+    g = torch.Generator().manual_seed(6)
+    xs = torch.randn(300, 128, generator=g) * torch.logspace(-6, 3, 300)[:, None]
+    xs[5] = 0.0
+    xs[6, :] = 1e-30
+    x = _bf16_bits(xs)
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).float()
+    amax = xf.abs().amax(dim=1).clamp(min=1e-4)
+    sc = amax / 448.0
+    codes = (xf / sc[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    kp, sp = oracle.act_quant_store(x, np.arange(300), 300)
+    assert np.array_equal(sp, sc.numpy())
+    assert np.array_equal(kp, codes)
+
+
+def test_act_quant_slots_and_error_bound():
+    g = torch.Generator().manual_seed(7)
+    xs = torch.randn(40, 128, generator=g) * 3
+    x = _bf16_bits(xs)
+    slot = np.array([(7 * t) % 64 for t in range(40)], np.int64)
+    slot[3] = -1            # not stored
+    slot[9] = 64            # outside the pool: not stored
+    kp0 = np.full((64, 128), 0xAB, np.uint8)
+    sp0 = np.full((64,), -7.0, np.float32)
+    kp, sp = oracle.act_quant_store(x, slot, 64, kp0.copy(), sp0.copy())
+    stored = {int(s) for s in slot if 0 <= s < 64}
+    for s in range(64):
+        if s not in stored:
+            assert np.all(kp[s] == 0xAB) and sp[s] == np.float32(-7.0)
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).double().numpy()
+    for t in range(40):
+        s = int(slot[t])
+        if not 0 <= s < 64:
+            continue
+        deq = oracle.e4m3_decode(kp[s]) * float(sp[s])
+        # e4m3 keeps 3 mantissa bits: half an ulp is 2^-4 relative, or 2^-10 * scale below 2^-6
+        assert np.all(np.abs(deq - xf[t]) <= 2.0 ** -4 * np.abs(xf[t]) + 2.0 ** -10 * float(sp[s]) + 1e-30)
