@@ -21,6 +21,11 @@ of the same workload's rows per step (rank 0 only).
 logits (fp8idx_mqa_logits, rows chunked so that one chunk of logits stays
 within 2 GiB) followed by fp8idx_topk_rows on each chunk, the loop of the
 pages' chunked benchmark.  Same metric, same algorithmic flops.
+
+--path act_quant (with --workload 4) times the producer of the paged keys:
+fp8idx_act_quant_store of every key of the workload's requests (bf16 rows
+to e4m3 codes and per-token scales, stored through the block table).  Its
+metric is HBM GB/s: 256 B read, 8 B of slot read and 132 B written per key.
 """
 from __future__ import annotations
 
@@ -54,8 +59,9 @@ def strict_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, choices=sorted(workloads.WORKLOADS), default=WORKLOAD,
                     help="workload index (default 1, the headline causal prefill)")
-    ap.add_argument("--path", choices=["fused", "chained"], default="fused",
-                    help="fused logits + top-k (default) or materialised logits then top-k")
+    ap.add_argument("--path", choices=["fused", "chained", "act_quant"], default="fused",
+                    help="fused logits + top-k (default), materialised logits then top-k, "
+                         "or the key quantisation into the paged pool (workload 4)")
     ap.add_argument("--quick", action="store_true",
                     help="device timing only: skip the end-to-end pass and the CPU baseline")
     a = ap.parse_args(argv)
@@ -63,6 +69,8 @@ def strict_args(argv=None):
         ap.error("need --gpus >= 1, --steps >= 1, --warmup >= 3")
     if a.path == "chained" and (a.workload == 4 or a.impl == "reference"):
         ap.error("--path chained is the prefill comparison path of our implementation")
+    if a.path == "act_quant" and (a.workload != 4 or a.impl == "reference"):
+        ap.error("--path act_quant fills the paged key pool of workload 4")
     return a
 
 
@@ -262,6 +270,29 @@ def make_case(fx, index, dev, path="fused"):
     """Device-resident inputs, outputs, workspace and the C-ABI call for one workload."""
     d = workloads.make_workload(index)
     topk = workloads.TOPK
+    if index == 4 and path == "act_quant":
+        # every key of every request, as bf16, into its slot of a fresh pool
+        L = d["seq_lens"].long()
+        bt = d["block_table"].long()
+        slot = torch.cat([bt[b, torch.arange(int(L[b])) // 64] * 64 + torch.arange(int(L[b])) % 64
+                          for b in range(d["B"])])
+        T = slot.numel()
+        g = torch.Generator().manual_seed(d["seed"] + 1000)
+        xk = (torch.randn(T, workloads.D, generator=g) * 2).to(torch.bfloat16)
+        host = {"x": xk.pin_memory(), "slot": slot.pin_memory()}
+        dv = {x: host[x].to(dev) for x in host}
+        P = d["P"]
+        out = torch.empty((P, 64, workloads.D), dtype=torch.uint8, device=dev)
+        sp = torch.empty((P, 64), dtype=torch.float32, device=dev)
+        out_host = torch.empty(out.shape, dtype=torch.uint8).pin_memory()
+
+        def call():
+            fx.act_quant_store(dv["x"], dv["slot"], out, sp)
+        return dict(d=d, call=call, host=host, dv=dv, out=out, out_host=out_host, ws=None, pairs=T,
+                    flops=0, bytes=T * (2 * workloads.D + 8 + workloads.D + 4),
+                    kernel="act_quant_store_kernel (bf16 keys -> e4m3 pool + scales)", bound="hbm",
+                    launches=1, metric="k-pool fp8 quantise+store GB/s (act_quant, workload 4 keys)",
+                    unit="GB/s")
     if index == 4:
         keys = ("q", "k_pages", "s_pages", "w", "block_table", "seq_lens")
         host = {x: d[x].pin_memory() for x in keys}
@@ -316,7 +347,7 @@ def make_case(fx, index, dev, path="fused"):
         launches = 2 if index in (0, 4) else 1  # + the merge kernel when the key axis is split
     return dict(d=d, call=call, host=host, dv=dv, out=out, out_host=out_host, ws=ws, pairs=pairs,
                 flops=FLOP_PER_PAIR * pairs, bytes=nbytes, kernel=kernel, bound=bound,
-                launches=launches)
+                launches=launches, metric=METRIC, unit=UNIT)
 
 
 def run_ours(args, rank, world, local, pg):
@@ -356,7 +387,8 @@ def run_ours(args, rank, world, local, pg):
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     total_ms = max_over_ranks(pg, sum(step_ms))
     ms_per_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    work = flops / 1e12 if case["unit"] == UNIT else case["bytes"] / 1e9  # per step, in the unit's terms
+    value = world * work * args.steps / (total_ms / 1e3)
     status = fx.read_device_status(ws)
     kstats = fx.read_device_stats(ws) if ws is not None else None  # counters of the last timed call
 
@@ -380,7 +412,7 @@ def run_ours(args, rank, world, local, pg):
         torch.cuda.synchronize(dev)
         barrier(pg)
         e2e_ms = max_over_ranks(pg, sum(a.elapsed_time(b) for a, b in zip(e_starts, e_ends)))
-        e2e_value = world * flops * args.steps / (e2e_ms / 1e3) / 1e12
+        e2e_value = world * work * args.steps / (e2e_ms / 1e3)
 
     if rank != 0:
         return None
@@ -398,9 +430,10 @@ def run_ours(args, rank, world, local, pg):
                 "frac": achieved / hbm_peak, "traffic": None,
                 "peak_source": f"{peak_src} HBM copy bandwidth", "algorithmic_bytes": case["bytes"]}
     roof["kernel"] = case["kernel"]
-    roof["traffic"] = measured_traffic(d["name"])  # bytes per launch, ncu record
+    # bytes per launch from the ncu record of the fused kernel (other paths have none)
+    roof["traffic"] = measured_traffic(d["name"]) if args.path == "fused" else None
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": case["metric"], "value": value, "unit": case["unit"], "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3", "data": "synthetic",
         "config": {"workload": d["name"], "H": workloads.H, "D": workloads.D, "topk": workloads.TOPK,
@@ -409,7 +442,7 @@ def run_ours(args, rank, world, local, pg):
                    "parallelism": f"replicas x{world} (one independent slice per GPU)"},
         "rows_keys_per_s": world * pairs * args.steps / (total_ms / 1e3),
         "roofline": roof,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": e2e_value, "unit": case["unit"], "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": None if e2e_ms is None else e2e_ms / args.steps},
         "gpu_launches": args.steps * case["launches"],
@@ -423,7 +456,7 @@ def run_ours(args, rank, world, local, pg):
             line["config"][key] = d[key]
     if args.path != "fused":
         line["config"]["path"] = args.path
-    if args.workload != 4 and not args.quick and args.path == "fused":
+    if args.workload != 4 and not args.quick and args.path == "fused":  # the oracle's own metric
         line["cpu_baseline"] = cpu_baseline(d)
     return line
 

@@ -10,6 +10,7 @@ PyTorch fallback, and a missing or unloadable library raises.
   topk_rows(logits, ks, ke, topk)                        -> idx [m, topk] i32
   mqa_logits_topk(q, k, s, w, ks, ke, topk)              -> idx (and values)
   paged_mqa_logits_topk(q, k_pages, s_pages, w, block_table, seq_lens, R, topk)
+  act_quant_store(x, slot_mapping, k_pages, s_pages)     bf16 keys -> fp8 key pool
 
 q/k are fp8 e4m3fn bytes (torch.uint8 or torch.float8_e4m3fn), s/w float32,
 ks/ke/block_table/seq_lens int32.
@@ -70,8 +71,10 @@ def lib() -> ctypes.CDLL:
             L.fp8idx_last_error.restype = ctypes.c_char_p
             L.fp8idx_num_sms.restype = ctypes.c_int
             L.fp8idx_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+            L.fp8idx_act_quant_store.argtypes = [vp, i64, i32, vp, i64, vp, vp, vp]
             for name in ("fp8idx_mqa_logits", "fp8idx_topk_rows", "fp8idx_mqa_logits_topk",
-                         "fp8idx_paged_mqa_logits_topk", "fp8idx_read_device_status"):
+                         "fp8idx_paged_mqa_logits_topk", "fp8idx_read_device_status",
+                         "fp8idx_act_quant_store"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -234,3 +237,26 @@ def paged_mqa_logits_topk(q, k_pages, s_pages, w, block_table, seq_lens, R: int,
                                               _ptr(out), _ptr(out_vals), _ptr(workspace),
                                               workspace.numel(), _stream(stream)))
     return (out, out_vals) if return_values else out
+
+
+def act_quant_store(x, slot_mapping, k_pages, s_pages, stream=None):
+    """Quantise bf16 key rows into the fp8 key pool, in place.
+
+    x [T, 128] bfloat16; slot_mapping [T] int64 (pool slot = page * 64 + row,
+    a slot outside the pool is skipped); k_pages [P, 64, 128] uint8 (or
+    float8_e4m3fn) and s_pages [P, 64] float32 receive the e4m3 codes and the
+    per-token scale max(max |x|, 1e-4) / 448.
+    """
+    if not isinstance(x, torch.Tensor) or x.dtype != torch.bfloat16:
+        raise TypeError("x must be a bfloat16 tensor")
+    x = _dev(x, "x")
+    slot_mapping = _dev(slot_mapping, "slot_mapping", torch.int64)
+    k_pages = _bytes(k_pages, "k_pages")
+    s_pages = _dev(s_pages, "s_pages", torch.float32)
+    T = x.shape[0]
+    num_slots = s_pages.numel()
+    if x.dim() != 2 or slot_mapping.numel() != T or k_pages.numel() != num_slots * x.shape[1]:
+        raise ValueError("x [T, D], slot_mapping [T], k_pages [slots, D] and s_pages [slots] disagree")
+    _check(lib().fp8idx_act_quant_store(_ptr(x), T, x.shape[1], _ptr(slot_mapping), num_slots,
+                                        _ptr(k_pages), _ptr(s_pages), _stream(stream)))
+    return k_pages, s_pages

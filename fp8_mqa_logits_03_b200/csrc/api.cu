@@ -25,6 +25,9 @@ __device__ int g_logits_status[kStatusBytes / 4];  // status block of the last f
 // address comes from cudaGetSymbolAddress.
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+cudaError_t launch_act_quant_store(const uint16_t* x, int64_t T, const int64_t* slot, int64_t num_slots,
+                                   uint8_t* k_pool, float* s_pool, cudaStream_t st);
 }
 
 namespace {
@@ -555,6 +558,20 @@ int fp8idx_read_device_stats(const void* ws, uint32_t* out, int count, void* str
   cudaError_t e = cudaMemcpyAsync(out, ws, sizeof(uint32_t) * count, cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "stats read");
+  return ok();
+}
+
+int fp8idx_act_quant_store(const uint16_t* x, int64_t T, int D, const int64_t* slot, int64_t num_slots,
+                           uint8_t* k_pool, float* s_pool, void* stream) {
+  if (D != kDim) return fail(FP8IDX_EUNSUPPORTED, "only D=128 is supported (got D=%d)", D);
+  if (T < 0 || num_slots < 0) return fail(FP8IDX_EINVAL, "negative size");
+  if (T > (int64_t(1) << 34)) return fail(FP8IDX_EINVAL, "T=%lld is too large", (long long)T);
+  if (T == 0) return ok();
+  if (!x || !slot || !k_pool || !s_pool) return fail(FP8IDX_EINVAL, "null pointer");
+  if (!aligned(x, 8) || !aligned(slot, 8) || !aligned(k_pool, 4) || !aligned(s_pool, 4))
+    return fail(FP8IDX_EINVAL, "x and slot must be 8-byte aligned, k_pool and s_pool 4-byte aligned");
+  cudaError_t e = launch_act_quant_store(x, T, slot, num_slots, k_pool, s_pool, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant_store launch");
   return ok();
 }
 

@@ -156,6 +156,26 @@ int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const flo
                                    float* out_vals, void* stream);
 
 /*
+ * Key quantisation into the paged key pool: the producer of k_pages /
+ * s_pages above (the `act_quant` step and the fp8 k-pool stores named on the
+ * "Serve GLM-5.3-Flash on SM80" page, commit notes).  The pages do not print
+ * the scale rule; the one taken is a per-token fp32 scale
+ *     s_t = max(max_d |x[t,d]|, 1e-4) / 448
+ * and codes e4m3(x[t,d] / s_t), rounded to nearest even and saturated at
+ * +-448, both computed in fp32.  Token t goes to pool slot slot[t]
+ * (physical page slot[t] / 64, row slot[t] % 64); a slot outside
+ * [0, num_slots) is skipped.
+ *   x       [T, D] bf16 bit patterns, D must be 128, 8-byte aligned
+ *   slot    [T] int64, 8-byte aligned
+ *   k_pool  [num_slots, 128] e4m3 bytes (k_pages viewed as slots), 4-byte aligned
+ *   s_pool  [num_slots] fp32 (s_pages viewed as slots), 4-byte aligned
+ * Slots not named by any token are left untouched; two tokens naming one
+ * slot race.  No workspace.
+ */
+int fp8idx_act_quant_store(const uint16_t* x, int64_t T, int D, const int64_t* slot, int64_t num_slots,
+                           uint8_t* k_pool, float* s_pool, void* stream);
+
+/*
  * Tests and diagnostics.  fp8idx_read_device_status synchronises `stream`
  * and copies the status word written by the last call that used workspace
  * `ws` (ws == NULL: the last fp8idx_mqa_logits call) into *status_out.

@@ -80,3 +80,16 @@ def test_paged_rejects(L):
 def test_workspace_queries_reject_bad_shapes(L):
     assert L.fp8idx_mqa_logits_topk_workspace(8, 100, 32, 128, 0) == 0
     assert L.fp8idx_paged_mqa_logits_topk_workspace(4, 3, 16, 32, 128, 2048) == 0
+
+
+def test_act_quant_store_rejects(L):
+    def call(x=FAKE, T=4, D=128, slot=FAKE, slots=64, kp=FAKE, sp=FAKE):
+        return L.fp8idx_act_quant_store(x, T, D, slot, slots, kp, sp, None)
+    assert call(D=64) == fx.EUNSUPPORTED
+    assert call(T=-1) == fx.EINVAL
+    assert call(slots=-1) == fx.EINVAL
+    assert call(x=None) == fx.EINVAL
+    assert call(slot=MIS) == fx.EINVAL          # int64 slots: 8-byte aligned
+    assert call(x=MIS) == fx.EINVAL             # 4 bf16 per lane: 8-byte aligned
+    assert call(kp=ctypes.c_void_p(4096 + 2)) == fx.EINVAL
+    assert call(T=0) == fx.OK

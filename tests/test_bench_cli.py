@@ -23,6 +23,8 @@ def test_defaults_are_the_headline_run():
     ["--gpus", "0"],
     ["--path", "chained", "--workload", "4"],      # the paged form has no chained path
     ["--path", "chained", "--impl", "reference"],
+    ["--path", "act_quant"],                       # the key pool belongs to workload 4
+    ["--path", "act_quant", "--workload", "4", "--impl", "reference"],
     ["--workload", "9"],
     ["--wark", "3"],                               # no prefix matching of options
 ])
