@@ -24,12 +24,17 @@
  * stays far below 2^53 units of 2^-18.  The head-weighted sum and the key
  * scale are applied in float64 in ascending head order.
  *
+ * It also restates the producer of the paged keys (the key quantisation
+ * into the fp8 pool, at the end of this file).
+ *
  * Parity pins (tests/test_oracle.py): the codec against torch's e4m3fn
  * cast and the rounding ties printed on the "Serve GLM-5.3-Flash on SM80"
  * page (unit-test commit notes); the dot against an int64 evaluation;
  * hand-computed tiny logits (tests/golden/); torch float64 einsum on small
  * shapes; brute-force top-k over all subsets; mask invariants; the paged
- * form against the prefill form on a gathered key array.
+ * form against the prefill form on a gathered key array; the key
+ * quantisation against the codec, its scale floor, torch's fp32 arithmetic
+ * with torch's e4m3fn cast, and the e4m3 error bound.
  */
 #define _GNU_SOURCE
 #include <math.h>
