@@ -63,7 +63,10 @@ def strict_args(argv=None):
                     help="fused logits + top-k (default), materialised logits then top-k, "
                          "or the key quantisation into the paged pool (workload 4)")
     ap.add_argument("--quick", action="store_true",
-                    help="device timing only: skip the end-to-end pass and the CPU baseline")
+                    help="device timing only: skip the end-to-end pass, the CPU baseline, the fp8 "
+                         "GEMM peak and the other workloads")
+    ap.add_argument("--suite", action="store_true",
+                    help="with --quick: still time the other workloads and the fp8 GEMM peak")
     a = ap.parse_args(argv)
     if a.gpus < 1 or a.steps < 1 or a.warmup < 3:
         ap.error("need --gpus >= 1, --steps >= 1, --warmup >= 3")
@@ -99,6 +102,10 @@ def measured_traffic(workload_name: str):
     return None if e is None else e["dram_read_bytes"] + e["dram_write_bytes"]
 
 
+NOMINAL_FP8_TFLOPS = 4500.0  # B200 dense fp8 datasheet figure (context only)
+NOMINAL_HBM_GBS = 8000.0      # B200 HBM3e datasheet figure (context only)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -106,6 +113,32 @@ def load_peaks():
             p = json.load(f)
         return float(p["bf16_tflops"]), float(p.get("hbm_gbs", 6650.0)), "measured"
     return 1590.0, 6650.0, "fallback"
+
+
+def measure_fp8_peak(dev, size: int = 8192, reps: int = 10):
+    """Dense e4m3 x e4m3 -> bf16 GEMM throughput of the library routine
+    torch._scaled_mm at size^3 (best of `reps`, CUDA events): a denominator
+    only, nothing of the indexer runs through it.  None if unavailable."""
+    try:
+        g = torch.Generator(device=dev).manual_seed(0)
+        a = torch.randn(size, size, device=dev, generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn(size, size, device=dev, generator=g).to(torch.float8_e4m3fn)
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        for _ in range(3):
+            torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return 2.0 * size ** 3 / (best / 1e3) / 1e12
+    except Exception as exc:  # pragma: no cover - depends on the torch build
+        print(f"fp8 peak measurement unavailable: {exc}", file=sys.stderr)
+        return None
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -350,6 +383,72 @@ def make_case(fx, index, dev, path="fused"):
                 launches=launches, metric=METRIC, unit=UNIT)
 
 
+def time_device(call, steps: int, warmup: int, flush, stream):
+    """Per-step device times (ms) of `call` with CUDA events on `stream`; L2 is
+    flushed (untimed) before every step."""
+    for _ in range(warmup):
+        call()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        call()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in zip(starts, ends)]
+
+
+def roofline_of(case, mean_s, peaks):
+    """The dominant kernel's achieved figure against its measured peak (and, as
+    context, against the nominal datasheet peak and the measured fp8 GEMM)."""
+    bf16_peak, hbm_peak, peak_src, fp8_meas = peaks
+    fp8_peak = 2.0 * bf16_peak  # measured bf16 burst x nominal fp8/bf16 ratio (4.5 / 2.25)
+    if case["bound"] == "tensor":
+        achieved = case["flops"] / mean_s / 1e12
+        r = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+             "frac": achieved / fp8_peak, "traffic": None,
+             "peak_source": f"{peak_src} bf16 burst {bf16_peak} TFLOP/s x 2 (fp8/bf16 nominal ratio)",
+             "frac_of_nominal_fp8": achieved / NOMINAL_FP8_TFLOPS}
+        if fp8_meas:
+            r["frac_of_measured_fp8_gemm"] = achieved / fp8_meas
+    else:
+        achieved = case["bytes"] / mean_s / 1e9
+        r = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+             "frac": achieved / hbm_peak, "traffic": None,
+             "peak_source": f"{peak_src} HBM copy bandwidth", "algorithmic_bytes": case["bytes"],
+             "frac_of_nominal_hbm": achieved / NOMINAL_HBM_GBS}
+    r["kernel"] = case["kernel"]
+    return r
+
+
+SUITE = [(0, "fused"), (2, "fused"), (3, "fused"), (4, "fused"), (4, "act_quant")]
+
+
+def run_suite(fx, dev, flush, stream, peaks, steps=10, warmup=3):
+    """Device time, throughput and roofline fraction of every other workload
+    (and of the key quantisation), each timed like the headline."""
+    out = {}
+    for index, path in SUITE:
+        case = make_case(fx, index, dev, path)
+        ms = time_device(case["call"], steps, warmup, flush, stream)
+        status = fx.read_device_status(case["ws"]) if case["ws"] is not None else 0
+        mean_s = statistics.mean(ms) / 1e3
+        roof = roofline_of(case, mean_s, peaks)
+        name = case["d"]["name"] + ("" if path == "fused" else f"+{path}")
+        out[name] = {"ms_per_step": statistics.mean(ms), "steps": steps, "warmup": warmup,
+                     "achieved": roof["achieved"], "unit": roof["unit"], "frac": roof["frac"],
+                     "bound": roof["bound"], "kernel": roof["kernel"], "device_status": status,
+                     "rows_keys_per_s": case["pairs"] / mean_s if path == "fused" else None}
+        for key in ("frac_of_nominal_fp8", "frac_of_nominal_hbm", "frac_of_measured_fp8_gemm"):
+            if key in roof:
+                out[name][key] = roof[key]
+        del case
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, local, pg):
     import fp8_mqa_logits_03_b200 as fx
     from fp8_mqa_logits_03_b200 import build
@@ -414,27 +513,27 @@ def run_ours(args, rank, world, local, pg):
         e2e_ms = max_over_ranks(pg, sum(a.elapsed_time(b) for a, b in zip(e_starts, e_ends)))
         e2e_value = world * work * args.steps / (e2e_ms / 1e3)
 
+    mean_s = statistics.mean(step_ms) / 1e3
+    roof = roofline_of(case, mean_s, load_peaks() + (None,))
+    metric, unit, launches = case["metric"], case["unit"], case["launches"]
+
+    # every rank takes the same steps: the suite runs everywhere, rank 0 reports it
+    suite = fp8_meas = None
+    if not args.quick or args.suite:
+        del case, call, dv, host, out, out_host, ws
+        torch.cuda.empty_cache()
+        fp8_meas = measure_fp8_peak(dev)
+        suite = run_suite(fx, dev, flush, stream, load_peaks() + (fp8_meas,))
+        barrier(pg)
     if rank != 0:
         return None
-    bf16_peak, hbm_peak, peak_src = load_peaks()
-    fp8_peak = 2.0 * bf16_peak  # measured bf16 burst x nominal fp8/bf16 ratio (4.5 / 2.25)
-    mean_s = statistics.mean(step_ms) / 1e3
-    if case["bound"] == "tensor":
-        achieved = flops / mean_s / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
-                "frac": achieved / fp8_peak, "traffic": None,
-                "peak_source": f"{peak_src} bf16 burst {bf16_peak} TFLOP/s x 2 (fp8/bf16 nominal ratio)"}
-    else:
-        achieved = case["bytes"] / mean_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": None,
-                "peak_source": f"{peak_src} HBM copy bandwidth", "algorithmic_bytes": case["bytes"]}
-    roof["kernel"] = case["kernel"]
+    if fp8_meas and roof["bound"] == "tensor":
+        roof["frac_of_measured_fp8_gemm"] = roof["achieved"] / fp8_meas
     # bytes per launch from the ncu record of the fused kernel (other paths have none)
     roof["traffic"] = measured_traffic(d["name"]) if args.path == "fused" else None
     line = {
-        "metric": case["metric"], "value": value, "unit": case["unit"], "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3", "data": "synthetic",
         "config": {"workload": d["name"], "H": workloads.H, "D": workloads.D, "topk": workloads.TOPK,
                    "seed": d["seed"], "valid_pairs": pairs,
@@ -442,15 +541,19 @@ def run_ours(args, rank, world, local, pg):
                    "parallelism": f"replicas x{world} (one independent slice per GPU)"},
         "rows_keys_per_s": world * pairs * args.steps / (total_ms / 1e3),
         "roofline": roof,
-        "e2e": {"value": e2e_value, "unit": case["unit"], "h2d_bytes_per_step": h2d,
+        "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": None if e2e_ms is None else e2e_ms / args.steps},
-        "gpu_launches": args.steps * case["launches"],
+        "gpu_launches": args.steps * launches,
         "clocks": clocks.summary(),
         "device_status": status,
         "kernel_stats": kstats,
         "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)},
     }
+    if fp8_meas:
+        line["fp8_tflops_measured"] = fp8_meas
+    if suite is not None:
+        line["workloads"] = suite
     for key in ("m", "n", "B", "R"):
         if key in d:
             line["config"][key] = d[key]

@@ -11,6 +11,8 @@ PyTorch fallback, and a missing or unloadable library raises.
   mqa_logits_topk(q, k, s, w, ks, ke, topk)              -> idx (and values)
   paged_mqa_logits_topk(q, k_pages, s_pages, w, block_table, seq_lens, R, topk)
   act_quant_store(x, slot_mapping, k_pages, s_pages)     bf16 keys -> fp8 key pool
+  prepare_ragged(seq_len, q_len, req_idx, req_to_token, q_cap)  ragged ks/ke (+ index copy)
+  topk_transform(idx, page_table, page_size, ...)        selected positions -> physical slots
 
 q/k are fp8 e4m3fn bytes (torch.uint8 or torch.float8_e4m3fn), s/w float32,
 ks/ke/block_table/seq_lens int32.
@@ -71,10 +73,14 @@ def lib() -> ctypes.CDLL:
             L.fp8idx_last_error.restype = ctypes.c_char_p
             L.fp8idx_num_sms.restype = ctypes.c_int
             L.fp8idx_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+            L.fp8idx_debug_withhold_first_tile.argtypes = [ctypes.c_int]
             L.fp8idx_act_quant_store.argtypes = [vp, i64, i32, vp, i64, vp, vp, vp]
+            L.fp8idx_prepare_ragged.argtypes = [vp, vp, vp, i32, vp, i64, i64, vp, vp, vp, i64, vp, i64,
+                                                vp]
+            L.fp8idx_topk_transform.argtypes = [vp, i64, i32, vp, vp, i32, vp, i64, i64, i32, vp, vp]
             for name in ("fp8idx_mqa_logits", "fp8idx_topk_rows", "fp8idx_mqa_logits_topk",
                          "fp8idx_paged_mqa_logits_topk", "fp8idx_read_device_status",
-                         "fp8idx_act_quant_store"):
+                         "fp8idx_act_quant_store", "fp8idx_prepare_ragged", "fp8idx_topk_transform"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -120,16 +126,33 @@ def set_wait_limit_ns(ns: int) -> None:
     lib().fp8idx_set_wait_limit_ns(int(ns))
 
 
+def debug_withhold_first_tile(on: bool) -> None:
+    """Tests only: later fused / paged calls never load their first key tile,
+    so a bounded wait runs out and the call reports WAIT_TIMEOUT."""
+    lib().fp8idx_debug_withhold_first_tile(1 if on else 0)
+
+
+# Names the library's fixed scratch array (the allocation-free entry point)
+# where a workspace is expected by the diagnostics calls.
+NOALLOC_WS = "noalloc"
+
+
+def _ws_ptr(workspace):
+    return ctypes.c_void_p(1) if isinstance(workspace, str) and workspace == NOALLOC_WS else _ptr(workspace)
+
+
 def read_device_status(workspace=None, stream=None) -> int:
+    """Status bits of the last call that used `workspace` (None: the last
+    mqa_logits call; NOALLOC_WS: the last allocation-free call).  Synchronises."""
     v = ctypes.c_int(0)
-    _check(lib().fp8idx_read_device_status(_ptr(workspace), ctypes.byref(v), _stream(stream)))
+    _check(lib().fp8idx_read_device_status(_ws_ptr(workspace), ctypes.byref(v), _stream(stream)))
     return v.value
 
 
 def read_device_stats(workspace, stream=None) -> dict:
     """Counters the fused top-k left in a workspace's status block (tuning aid)."""
     buf = (ctypes.c_uint32 * 5)()
-    _check(lib().fp8idx_read_device_stats(_ptr(workspace), buf, 5, _stream(stream)))
+    _check(lib().fp8idx_read_device_stats(_ws_ptr(workspace), buf, 5, _stream(stream)))
     return dict(status=buf[0], compactions=buf[1], general_selects=buf[2], candidates=buf[3],
                 max_boundary=buf[4])
 
@@ -260,3 +283,51 @@ def act_quant_store(x, slot_mapping, k_pages, s_pages, stream=None):
     _check(lib().fp8idx_act_quant_store(_ptr(x), T, x.shape[1], _ptr(slot_mapping), num_slots,
                                         _ptr(k_pages), _ptr(s_pages), _stream(stream)))
     return k_pages, s_pages
+
+
+# ---------------------------------------------------------------------------- index preparation
+
+def prepare_ragged(seq_len, q_len, req_idx, req_to_token, q_cap: int, ragged_cap: int = 0,
+                   with_ragged: bool = True, ks=None, ke=None, row_table=None, ragged=None, stream=None):
+    """Ragged key ranges of the batch's query rows (and its ragged token-slot
+    buffer): fp8idx_prepare_ragged.  Returns (ks, ke, row_table, ragged or None)."""
+    seq_len = _dev(seq_len, "seq_len", torch.int32)
+    q_len = _dev(q_len, "q_len", torch.int32)
+    req_idx = _dev(req_idx, "req_idx", torch.int32)
+    req_to_token = _dev(req_to_token, "req_to_token", torch.int32)
+    if req_to_token.dim() != 2:
+        raise ValueError("req_to_token must be [rows, ld]")
+    B = seq_len.numel()
+    if q_len.numel() != B or req_idx.numel() != B:
+        raise ValueError("seq_len, q_len and req_idx must have one entry per request")
+    dev = seq_len.device
+    ks = torch.empty(q_cap, dtype=torch.int32, device=dev) if ks is None else ks
+    ke = torch.empty(q_cap, dtype=torch.int32, device=dev) if ke is None else ke
+    row_table = torch.empty(q_cap, dtype=torch.int32, device=dev) if row_table is None else row_table
+    if with_ragged and ragged is None:
+        ragged = torch.empty(ragged_cap, dtype=torch.int32, device=dev)
+    _check(lib().fp8idx_prepare_ragged(_ptr(seq_len), _ptr(q_len), _ptr(req_idx), B, _ptr(req_to_token),
+                                       req_to_token.shape[0], req_to_token.stride(0), _ptr(ks), _ptr(ke),
+                                       _ptr(row_table), q_cap, _ptr(ragged) if with_ragged else None,
+                                       ragged.numel() if with_ragged else 0, _stream(stream)))
+    return ks, ke, row_table, (ragged if with_ragged else None)
+
+
+def topk_transform(idx, page_table, page_size: int = 1, row_base=None, row_table=None,
+                   rows_per_table_row: int = 1, out=None, stream=None):
+    """Selected positions -> physical slots through a page table
+    (fp8idx_topk_transform); -1 stays -1.  out may be idx (in place)."""
+    idx = _dev(idx, "idx", torch.int32)
+    page_table = _dev(page_table, "page_table", torch.int32)
+    if idx.dim() != 2 or page_table.dim() != 2:
+        raise ValueError("idx must be [rows, topk] and page_table [rows, ld]")
+    rows, k = idx.shape
+    if row_base is not None:
+        row_base = _dev(row_base, "row_base", torch.int32)
+    if row_table is not None:
+        row_table = _dev(row_table, "row_table", torch.int32)
+    out = torch.empty_like(idx) if out is None else out
+    _check(lib().fp8idx_topk_transform(_ptr(idx), rows, k, _ptr(row_base), _ptr(row_table),
+                                       rows_per_table_row, _ptr(page_table), page_table.shape[0],
+                                       page_table.stride(0), page_size, _ptr(out), _stream(stream)))
+    return out

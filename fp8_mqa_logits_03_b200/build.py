@@ -8,7 +8,7 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp8idx.so")
-SOURCES = ["kernels.cu", "quant.cu", "api.cu"]
+SOURCES = ["kernels.cu", "quant.cu", "index_prep.cu", "api.cu"]
 DEPS = SOURCES + ["kernels.cuh", "ptx.cuh", "select.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "fp8idx.h")
 

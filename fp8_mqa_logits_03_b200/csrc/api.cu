@@ -28,6 +28,15 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 cudaError_t launch_act_quant_store(const uint16_t* x, int64_t T, const int64_t* slot, int64_t num_slots,
                                    uint8_t* k_pool, float* s_pool, cudaStream_t st);
+constexpr int kMaxPrepBatch = 8192;
+cudaError_t launch_prepare_ragged(const int32_t* seq_len, const int32_t* q_len, const int32_t* req_idx, int B,
+                                  const int32_t* table, int64_t table_rows, int64_t ld, int32_t* ks, int32_t* ke,
+                                  int32_t* row_table, int64_t q_cap, int32_t* ragged, int64_t ragged_cap,
+                                  int sms, cudaStream_t st);
+cudaError_t launch_topk_transform(const int32_t* idx, int64_t rows, int topk, const int32_t* row_base,
+                                  const int32_t* row_table, int rows_per_table_row, const int32_t* table,
+                                  int64_t table_rows, int64_t ld, int page_size, int32_t* out, int sms,
+                                  cudaStream_t st);
 }
 
 namespace {
@@ -36,6 +45,7 @@ using namespace fp8idx;
 
 thread_local std::string t_last_error;
 unsigned long long g_wait_limit_ns = 2000000000ull;
+int g_debug_withhold = 0;
 
 int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 int fail(int code, const char* fmt, ...) {
@@ -117,19 +127,21 @@ struct Plan {
   size_t off_cand = 0, off_scratch = 0, off_part = 0, off_cnt = 0, off_theta = 0, total = 0;
 };
 
-// Room for the candidates a row collects over `keys` keys.  With a running
-// threshold at the k-th value seen so far, a key enters with probability
-// about min(1, k / position), so about k * (1 + ln(keys / k)) keys enter in
-// all; half again of that covers the histogram's bin slack.  Overflow is
-// still handled (an exact compaction in the kernel), only slower.
+// Room for the candidates a row collects over `keys` keys (four equal
+// segments, one per epilogue warp of the row).  With a running threshold at
+// the k-th value seen so far, a key enters with probability about
+// min(1, k / position), so about k * (1 + ln(keys / k)) keys enter in all;
+// half again of that covers the histogram's bin slack.  A segment that fills
+// up is compacted to its exact top-k in the kernel, so it must hold k plus
+// the 32 keys per tile its warp may append before the next vote; a segment
+// never needs more than its whole share of the keys (32 per tile).
 int candidate_capacity(int topk, int64_t keys) {
   const double ratio = std::max(1.0, static_cast<double>(keys) / topk);
   const double expect = topk * (1.0 + std::log(ratio));
   const int64_t cap = static_cast<int64_t>(1.5 * expect) + 2 * kBlockKeys;
-  // Each of the row's four segments must hold its share of the k kept by a
-  // compaction plus the 32 keys per tile a warp may add between two votes.
-  const int64_t floor_cap = 2 * static_cast<int64_t>(topk) + 4 * (kMaxVoteTiles + 2) * 32;
-  return static_cast<int>(round_up(std::max<int64_t>(cap, floor_cap), kBlockKeys));
+  const int64_t floor_cap = 4 * (static_cast<int64_t>(topk) + kMaxVoteTiles * 32);
+  const int64_t all_keys = round_up(std::max<int64_t>(keys, 1), kBlockKeys);
+  return static_cast<int>(round_up(std::min(all_keys, std::max<int64_t>(cap, floor_cap)), kBlockKeys));
 }
 
 void finish_plan(Plan& pl, int64_t groups, int sms, int topk, int64_t axis) {
@@ -202,6 +214,46 @@ int check_topk(int topk) {
   return FP8IDX_OK;
 }
 
+// Device address of the no-alloc scratch array on the current device,
+// looked up once per device index (under a lock) and kept for the process.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "current device");
+  constexpr int kMaxDevices = 64;
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP8IDX_EUNSUPPORTED, "device index %d out of range", dev);
+  static std::mutex mu;
+  static void* scratch_of[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (!scratch_of[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "no-alloc scratch address");
+    scratch_of[dev] = ptr;
+  }
+  *out = scratch_of[dev];
+  return FP8IDX_OK;
+}
+
+// A workspace argument of the diagnostics calls: NULL names the logits
+// status block, FP8IDX_NOALLOC_WS the no-alloc scratch array.
+int resolve_status_source(const void* ws, const void** src) {
+  if (ws == FP8IDX_NOALLOC_WS) {
+    void* p = nullptr;
+    const int rc = noalloc_scratch(&p);
+    if (rc != FP8IDX_OK) return rc;
+    *src = p;
+  } else if (!ws) {
+    void* sym = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&sym, g_logits_status);
+    if (e != cudaSuccess) return cuda_fail(e, "status symbol");
+    *src = sym;
+  } else {
+    *src = ws;
+  }
+  return FP8IDX_OK;
+}
+
 #define FP8IDX_TRY(x)          \
   do {                         \
     int _rc = (x);             \
@@ -234,6 +286,8 @@ const char* fp8idx_last_error(void) { return t_last_error.c_str(); }
 int fp8idx_num_sms(void) { return device_sms(); }
 
 void fp8idx_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
+
+void fp8idx_debug_withhold_first_tile(int on) { g_debug_withhold = on ? 1 : 0; }
 
 int fp8idx_mqa_logits(const uint8_t* q, const uint8_t* k, const float* s, const float* w,
                       const int32_t* ks, const int32_t* ke, int64_t m, int64_t n, int H, int D,
@@ -273,6 +327,7 @@ int fp8idx_mqa_logits(const uint8_t* q, const uint8_t* k, const float* s, const 
   if (e != cudaSuccess) return cuda_fail(e, "status reset");
   p.status = status;
   p.wait_limit_ns = g_wait_limit_ns;
+  p.debug_withhold_first_tile = g_debug_withhold;
   e = launch_indexer_prefill_logits(p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "mqa_logits launch");
   return ok();
@@ -355,6 +410,7 @@ int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, c
     if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
   }
   p.wait_limit_ns = g_wait_limit_ns;
+  p.debug_withhold_first_tile = g_debug_withhold;
   e = launch_indexer_prefill_topk(p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "mqa_logits_topk launch");
   if (pl.n_chunks > 1) {
@@ -443,6 +499,7 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
     if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
   }
   p.wait_limit_ns = g_wait_limit_ns;
+  p.debug_withhold_first_tile = g_debug_withhold;
   e = launch_indexer_paged_topk(p, R, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "paged_mqa_logits_topk launch");
   if (pl.n_chunks > 1) {
@@ -477,24 +534,9 @@ int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const flo
   if (m == 0) return ok();
   if (!out_idx || !aligned(out_idx, 4) || !aligned(out_vals, 4))
     return fail(FP8IDX_EINVAL, "out_idx must be non-null; outputs 4-byte aligned");
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "current device");
-  constexpr int kMaxDevices = 64;
-  if (dev < 0 || dev >= kMaxDevices) return fail(FP8IDX_EUNSUPPORTED, "device index %d out of range", dev);
-  static std::mutex mu;
-  static void* scratch_of[kMaxDevices] = {};
   void* scratch = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    if (!scratch_of[dev]) {
-      void* ptr = nullptr;
-      e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-      if (e != cudaSuccess) return cuda_fail(e, "no-alloc scratch address");
-      scratch_of[dev] = ptr;
-    }
-    scratch = scratch_of[dev];
-  }
+  FP8IDX_TRY(noalloc_scratch(&scratch));
+  cudaError_t e;
   int sms = device_sms();
   if (sms <= 0) return fail(FP8IDX_ECUDA, "no CUDA device");
   Plan pl;
@@ -542,6 +584,7 @@ int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const flo
     if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
   }
   p.wait_limit_ns = g_wait_limit_ns;
+  p.debug_withhold_first_tile = g_debug_withhold;
   e = launch_indexer_prefill_topk(p, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "mqa_logits_topk_noalloc launch");
   if (pl.n_chunks > 1) {
@@ -553,9 +596,11 @@ int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const flo
 }
 
 int fp8idx_read_device_stats(const void* ws, uint32_t* out, int count, void* stream) {
-  if (!ws || !out || count < 1 || count > kStatusBytes / 4) return fail(FP8IDX_EINVAL, "bad arguments");
+  if (!out || count < 1 || count > kStatusBytes / 4) return fail(FP8IDX_EINVAL, "bad arguments");
+  const void* src = nullptr;
+  FP8IDX_TRY(resolve_status_source(ws, &src));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemcpyAsync(out, ws, sizeof(uint32_t) * count, cudaMemcpyDeviceToHost, st);
+  cudaError_t e = cudaMemcpyAsync(out, src, sizeof(uint32_t) * count, cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "stats read");
   return ok();
@@ -575,16 +620,58 @@ int fp8idx_act_quant_store(const uint16_t* x, int64_t T, int D, const int64_t* s
   return ok();
 }
 
+int fp8idx_prepare_ragged(const int32_t* seq_len, const int32_t* q_len, const int32_t* req_idx, int B,
+                          const int32_t* req_to_token, int64_t table_rows, int64_t ld_table, int32_t* ks,
+                          int32_t* ke, int32_t* row_table, int64_t q_cap, int32_t* ragged, int64_t ragged_cap,
+                          void* stream) {
+  if (B < 0 || B > kMaxPrepBatch) return fail(FP8IDX_EINVAL, "B must be in [0, %d] (got %d)", kMaxPrepBatch, B);
+  if (q_cap < 0 || ragged_cap < 0 || table_rows < 0 || ld_table < 0)
+    return fail(FP8IDX_EINVAL, "negative size");
+  if (q_cap > INT32_MAX || ragged_cap > INT32_MAX)
+    return fail(FP8IDX_EINVAL, "capacities must stay below 2^31 (int32 key positions)");
+  if (q_cap == 0 && (!ragged || ragged_cap == 0)) return ok();
+  if ((B > 0 && (!seq_len || !q_len || !req_idx)) || (q_cap > 0 && (!ks || !ke)))
+    return fail(FP8IDX_EINVAL, "null seq_len, q_len, req_idx, ks or ke");
+  if (ragged && ragged_cap > 0 && table_rows > 0 && !req_to_token) return fail(FP8IDX_EINVAL, "null req_to_token");
+  if (!aligned(seq_len, 4) || !aligned(q_len, 4) || !aligned(req_idx, 4) || !aligned(req_to_token, 4) ||
+      !aligned(ks, 4) || !aligned(ke, 4) || !aligned(row_table, 4) || !aligned(ragged, 4))
+    return fail(FP8IDX_EINVAL, "pointers must be 4-byte aligned");
+  const int sms = device_sms();
+  if (sms <= 0) return fail(FP8IDX_ECUDA, "no CUDA device");
+  cudaError_t e = launch_prepare_ragged(seq_len, q_len, req_idx, B, req_to_token, table_rows, ld_table, ks, ke,
+                                        row_table, q_cap, ragged, ragged ? ragged_cap : 0, sms,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prepare_ragged launch");
+  return ok();
+}
+
+int fp8idx_topk_transform(const int32_t* idx, int64_t rows, int topk, const int32_t* row_base,
+                          const int32_t* row_table, int rows_per_table_row, const int32_t* page_table,
+                          int64_t table_rows, int64_t ld_table, int page_size, int32_t* out, void* stream) {
+  if (rows < 0 || topk < 0 || table_rows < 0 || ld_table < 0) return fail(FP8IDX_EINVAL, "negative size");
+  if (page_size < 1) return fail(FP8IDX_EINVAL, "page_size must be >= 1 (got %d)", page_size);
+  if (!row_table && rows_per_table_row < 1)
+    return fail(FP8IDX_EINVAL, "rows_per_table_row must be >= 1 without row_table");
+  if (rows == 0 || topk == 0) return ok();
+  if (!idx || !out || (table_rows > 0 && ld_table > 0 && !page_table))
+    return fail(FP8IDX_EINVAL, "null idx, out or page_table");
+  if (!aligned(idx, 4) || !aligned(out, 4) || !aligned(row_base, 4) || !aligned(row_table, 4) ||
+      !aligned(page_table, 4))
+    return fail(FP8IDX_EINVAL, "pointers must be 4-byte aligned");
+  const int sms = device_sms();
+  if (sms <= 0) return fail(FP8IDX_ECUDA, "no CUDA device");
+  cudaError_t e = launch_topk_transform(idx, rows, topk, row_base, row_table, rows_per_table_row, page_table,
+                                        table_rows, ld_table, page_size, out, sms,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "topk_transform launch");
+  return ok();
+}
+
 int fp8idx_read_device_status(const void* ws, int* status_out, void* stream) {
   if (!status_out) return fail(FP8IDX_EINVAL, "null status_out");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const void* src = ws;
-  if (!src) {
-    void* sym = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&sym, g_logits_status);
-    if (e != cudaSuccess) return cuda_fail(e, "status symbol");
-    src = sym;
-  }
+  const void* src = nullptr;
+  FP8IDX_TRY(resolve_status_source(ws, &src));
   int v = 0;
   cudaError_t e = cudaMemcpyAsync(&v, src, sizeof(int), cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);

@@ -65,24 +65,39 @@ constexpr int kUpCap = kMaxTopK; // per select warp: keys above the boundary bin
 constexpr int kAtCap = 1024;     // per select warp: keys inside the boundary bin
 constexpr int kSelBatch = 16;    // candidate loads in flight per select thread
 
-// Per (slot, row) streaming state of the fused top-k.  A row's candidate
-// buffer holds four equal segments, one per TMEM lane quadrant (key block of
-// 32 inside each tile), so each epilogue warp appends with a private counter.
+// Per (slot, row) streaming state of the fused top-k, shared by the four
+// epilogue warps that own the row's keys.  A row's candidate buffer holds
+// four equal segments, one per TMEM lane quadrant (key block of 32 inside
+// each tile), so each warp appends with a private counter and needs no
+// barrier: the histogram is counted with shared-memory atomics, the window is
+// opened once by compare-and-swap, and the threshold only grows (atomicMax).
 struct RowState {
-  int wcnt[4];     // candidates in each segment
-  uint32_t theta;  // keep a key only if order_key >= theta
-  float theta_f;   // the float whose order key is theta (-inf when theta admits all)
-  uint32_t base;   // histogram window: bin = min((key - base) >> shift, kNB - 1)
-  int shift;
-  int mode;        // 0: window not set yet, 1: histogram live
-  uint32_t tmin;   // min / max key collected while the window is not set
-  uint32_t tmax;
-  int lo, hi;      // the row's key range inside this unit's chunk
-  int pad[2];
+  int wcnt[4];       // candidates in each segment (written when the unit ends)
+  uint32_t theta;    // lower bound on the row's k-th order key: keep a key iff key >= theta
+  int lo, hi;        // the row's key range inside this unit's chunk
+  int pad;
+  unsigned long long win;  // histogram window: base | shift << 32 | 1 << 40 once open
 };
+
+// Order key of a logit computed as fma(sum, scale, +0), which is -0 only when
+// a nonzero negative product rounds to zero: that -0 then orders just below
+// +0, as its exact value does.  Two instructions, no -0 fix-up.
+__device__ __forceinline__ uint32_t order_key_nz(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return b ^ (static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) | 0x80000000u);
+}
 
 __device__ __forceinline__ float theta_float(uint32_t key) {
   return key <= 0x007FFFFFu ? -INFINITY : key_to_float(key);
+}
+
+struct Window {
+  bool open;
+  uint32_t base;  // bin = min((key - base) >> shift, kNB - 1) for key >= base
+  int shift;
+};
+__device__ __forceinline__ Window window_of(unsigned long long w) {
+  return Window{(w >> 40) != 0, static_cast<uint32_t>(w), static_cast<int>((w >> 32) & 0xFF)};
 }
 
 struct SlotMeta {
@@ -168,21 +183,19 @@ __device__ __forceinline__ Unit get_unit(const IndexerParams& p, int u) {
 
 // Bounded wait on an mbarrier phase.  Gives up when another role has
 // aborted or after `limit_ns`, flagging the device status; never traps.
-// SLEEP backs off with nanosleep (long waits of idle roles, which then take
-// no issue slots from the epilogue); otherwise it spins (latency-critical
-// hand-offs) and looks at the clock only every 64 polls.
-template <bool SLEEP>
+// NAP_NS == 0 polls with try_wait (for the epilogue's own hand-offs, where
+// the phase is normally complete already); NAP_NS > 0 tests the phase and
+// sleeps NAP_NS between tests, so that a role that is ahead of the epilogue
+// (MMA issue, TMA producer, idle select warps) takes few issue slots from it.
+// The abort flag and the clock are looked at every 8 polls.
+template <uint32_t NAP_NS>
 __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                        int* status, unsigned long long limit_ns) {
   const uint64_t t0 = global_timer_ns();
-  uint32_t ns = 64;
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (SLEEP) {
-      __nanosleep(ns);
-      if (ns < 2048) ns <<= 1;
-    }
-    if (SLEEP || (it & 63) == 0) {
+    if (NAP_NS == 0 ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity)) return true;
+    if (NAP_NS) __nanosleep(NAP_NS);
+    if ((it & 7) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
@@ -193,11 +206,26 @@ __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volatile 
   }
 }
 
-template <bool SLEEP>
+// Nap lengths (ns) by role: the epilogue polls; the MMA thread naps briefly
+// (it has slack against the epilogue but must not delay the next tile); the
+// producer runs stages ahead; idle roles sleep long.
+#ifndef FP8IDX_NAP_MMA_NS
+#define FP8IDX_NAP_MMA_NS 64
+#endif
+#ifndef FP8IDX_NAP_PRODUCER_NS
+#define FP8IDX_NAP_PRODUCER_NS 256
+#endif
+#ifndef FP8IDX_NAP_IDLE_NS
+#define FP8IDX_NAP_IDLE_NS 2048
+#endif
+constexpr uint32_t kSpin = 0, kNap = FP8IDX_NAP_MMA_NS, kProd = FP8IDX_NAP_PRODUCER_NS,
+                   kSleep = FP8IDX_NAP_IDLE_NS;
+
+template <uint32_t NAP_NS>
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                            int* status, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  return wait_slow<SLEEP>(bar, parity, abort_flag, status, limit_ns);
+  return wait_slow<NAP_NS>(bar, parity, abort_flag, status, limit_ns);
 }
 
 // Uniform OR over the threads of a named barrier.
@@ -255,17 +283,16 @@ __device__ __forceinline__ float relu_dot32_x2(const uint32_t (&x)[32], const fl
   return ((l0 + ab0) + (l1 + ab1)) + ((l2 + ab2) + (l3 + ab3));
 }
 
-// Histogram slot of bin b: lane (b >> 4) owns bins [16 lane, 16 lane + 16),
-// stored transposed so that a warp reading one bin per lane hits 32 banks.
-__device__ __forceinline__ int hist_index(int b) { return (b & 15) * 32 + (b >> 4); }
-
 // (Only meaningful for key >= base; any other key maps to some bin in range.)
 __device__ __forceinline__ int hist_bin(uint32_t key, uint32_t base, int shift) {
   return static_cast<int>(min((key - base) >> shift, static_cast<uint32_t>(kNB - 1)));
 }
 
 // Find the boundary bin: the highest bin b such that at least k counted
-// candidates lie in bins >= b.  Every lane returns the same result.
+// candidates lie in bins >= b.  Every lane returns the same result.  The
+// histogram is stored plainly (bin b at h[b]); lane l reads bins 32 i + l,
+// so the 16 reads are conflict-free, and the search runs over the 16 rows
+// of 32 bins from the top, then over the lanes of the row that holds it.
 struct Boundary {
   bool found;
   int bin;
@@ -274,42 +301,36 @@ struct Boundary {
 };
 
 __device__ __forceinline__ Boundary find_boundary(const uint32_t* h, uint32_t k, int lane) {
-  uint32_t c[16];
-  uint32_t tot = 0;
+  constexpr int kRows = kNB / 32;
+  uint32_t c[kRows];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    c[i] = h[i * 32 + lane];
-    tot += c[i];
+  for (int i = 0; i < kRows; ++i) c[i] = h[i * 32 + lane];
+  Boundary B{false, 0, 0, 0};
+  uint32_t run = 0, above_row = 0, v = 0;
+  int bi = -1;
+#pragma unroll
+  for (int i = kRows - 1; i >= 0; --i) {
+    const uint32_t tot = __reduce_add_sync(0xFFFFFFFFu, c[i]);
+    const bool hit = bi < 0 && run + tot >= k;
+    above_row = hit ? run : above_row;
+    v = hit ? c[i] : v;
+    bi = hit ? i : bi;
+    run += tot;
   }
-  uint32_t suf = tot;
+  if (bi < 0) return B;
+  // inclusive suffix sum over lanes >= lane of the row's counts
+  uint32_t suf = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const uint32_t t = __shfl_down_sync(0xFFFFFFFFu, suf, off);
     if (lane + off < 32) suf += t;
   }
-  Boundary B{false, 0, 0, 0};
-  const uint32_t ball = __ballot_sync(0xFFFFFFFFu, suf >= k);
-  if (ball == 0) return B;
+  const uint32_t ball = __ballot_sync(0xFFFFFFFFu, above_row + suf >= k);
   const int ls = 31 - __clz(static_cast<int>(ball));
-  // inside lane ls: the highest of its 16 bins where the running count from
-  // the top reaches k (predicated, no divergent loop)
-  uint32_t run = suf - tot;
-  int bin = 0;
-  uint32_t above = 0, inbin = 0;
-  bool done = false;
-#pragma unroll
-  for (int i = 15; i >= 0; --i) {
-    const bool hit = !done && run + c[i] >= k;
-    bin = hit ? lane * 16 + i : bin;
-    inbin = hit ? c[i] : inbin;
-    above = hit ? run : above;
-    done = done || hit;
-    run += c[i];
-  }
   B.found = true;
-  B.bin = __shfl_sync(0xFFFFFFFFu, bin, ls);
-  B.above = __shfl_sync(0xFFFFFFFFu, above, ls);
-  B.inbin = __shfl_sync(0xFFFFFFFFu, inbin, ls);
+  B.bin = bi * 32 + ls;
+  B.inbin = __shfl_sync(0xFFFFFFFFu, v, ls);
+  B.above = above_row + __shfl_sync(0xFFFFFFFFu, suf, ls) - B.inbin;
   return B;
 }
 
@@ -383,7 +404,8 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
     }
     return cnt;
   }
-  if (FAST && st.mode == 1) {
+  const Window win = window_of(st.win);
+  if (FAST && win.open) {
     const Boundary B = find_boundary(h, static_cast<uint32_t>(k), lane);
     if (B.found) {
       if (g.tid == 0) atomicMax(reinterpret_cast<unsigned*>(stats + kStatMaxBoundary), B.inbin);
@@ -395,8 +417,8 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
       // the bin iff key >= hi_key (never when the bin is the top, clamped one).
       // (The bin holds at least one key, so its lower edge is below 2^32.)
       const uint32_t lo_key = static_cast<uint32_t>(
-          min(static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin) << st.shift), static_cast<uint64_t>(0xFFFFFFFFu)));
-      const uint64_t hi64 = static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin + 1) << st.shift);
+          min(static_cast<uint64_t>(win.base) + (static_cast<uint64_t>(B.bin) << win.shift), static_cast<uint64_t>(0xFFFFFFFFu)));
+      const uint64_t hi64 = static_cast<uint64_t>(win.base) + (static_cast<uint64_t>(B.bin + 1) << win.shift);
       const bool has_hi = B.bin < kNB - 1 && hi64 <= 0xFFFFFFFFull;
       const uint32_t hi_key = has_hi ? static_cast<uint32_t>(hi64) : 0xFFFFFFFFu;
 #pragma unroll
@@ -504,6 +526,143 @@ __device__ void write_row_topk(const IndexerParams& p, const SlotMeta& meta, int
   }
 }
 
+// ------------------------------------------------------------------ vote-time row maintenance
+//
+// The epilogue's hot loop only filters and appends.  Every few tiles each
+// warp, on its own schedule (no barrier), counts its newly appended
+// candidates into the rows' shared histograms, makes room in a segment that
+// is filling up, and reloads the rows' thresholds; warp qd of a warpgroup
+// also raises the threshold of the group's row qd from that row's histogram.
+// Each counted key is a real key of the row, so a histogram count taken at
+// any moment (other warps may still be adding) is a lower bound and the
+// threshold it gives stays a valid lower bound on the row's k-th value.
+
+__device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned long long* p) {
+  return *reinterpret_cast<const volatile unsigned long long*>(p);
+}
+__device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t* p) {
+  return *reinterpret_cast<const volatile uint32_t*>(p);
+}
+
+// Count candidates [from, to) of one warp's segment of a row into the row's
+// histogram.  If the row's window is not open yet (then from == 0: nothing of
+// this warp has been counted), the warp proposes one from its own candidates
+// (twice their key span above their minimum) by compare-and-swap; the first
+// proposal wins and every warp counts with it.  Returns the new counted mark.
+__device__ __forceinline__ int fold_segment(const uint2* seg, int from, int to, RowState* st, uint32_t* h,
+                                         int lane) {
+  if (from >= to) return from;
+  __syncwarp();  // the warp's own appends are visible to all its lanes
+  unsigned long long wv = ld_volatile_u64(&st->win);
+  if (!(wv >> 40)) {
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0;
+    for (int e = lane; e < to; e += 32) {
+      const uint32_t key = seg[e].x;
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+    }
+    kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+    kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+    const uint64_t span = static_cast<uint64_t>(kmax - kmin);
+    const int bits = 64 - __clzll(static_cast<long long>(2 * span + 1));
+    const int shift = bits > 9 ? bits - 9 : 0;
+    const unsigned long long mine =
+        static_cast<unsigned long long>(kmin) | (static_cast<unsigned long long>(shift) << 32) | (1ull << 40);
+    if (lane == 0) atomicCAS(&st->win, 0ull, mine);
+    __syncwarp();
+    wv = ld_volatile_u64(&st->win);
+  }
+  const Window w = window_of(wv);
+  for (int e0 = from; e0 < to; e0 += 4 * 32) {
+    uint32_t key[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = e0 + i * 32 + lane;
+      key[i] = e < to ? seg[e].x : 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = e0 + i * 32 + lane;
+      if (e < to && key[i] >= w.base) atomicAdd(&h[hist_bin(key[i], w.base, w.shift)], 1u);
+    }
+  }
+  return to;
+}
+
+// A contiguous candidate list as a select source.
+struct ListSrc {
+  const uint2* a;
+  int n;
+  __device__ __forceinline__ bool get(int e, uint64_t& K) const {
+    if (e >= n) return false;
+    const uint2 v = a[e];
+    K = compose_key(v.x, v.y);
+    return true;
+  }
+};
+
+// Make room in one warp's segment of a row (cnt candidates, all counted):
+// drop candidates below the row's threshold; if that leaves fewer than
+// `room` free slots, keep the segment's exact top-k, staged through `scr`.
+// The k-th kept key is then a lower bound on the row's k-th value, and,
+// since every later key has a larger index, a later key equal to it can
+// never enter the top-k: the threshold rises to just above it.  The
+// histogram keeps counting the dropped keys: they are real keys of the row.
+__device__ __forceinline__ int compact_segment(uint2* seg, int cnt, int room, int wcap, int k, RowState* st,
+                                            uint2* scr, const Group<1>& grp, int* stats, int lane) {
+  const uint32_t lt = (1u << lane) - 1u;
+  const uint32_t th = ld_volatile_u32(&st->theta);
+  __syncwarp();
+  int n = 0;
+  for (int e0 = 0; e0 < cnt; e0 += 32) {
+    const int e = e0 + lane;
+    const uint2 v = e < cnt ? seg[e] : make_uint2(0u, 0u);
+    const bool keep = e < cnt && v.x >= th;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, keep);
+    if (keep) seg[n + __popc(m & lt)] = v;  // n + rank <= e: never ahead of the reads
+    n += __popc(m);
+  }
+  __syncwarp();
+  if (n + room <= wcap) return n;
+  const ListSrc src{seg, n};
+  const SelectResult sel = group_select<1>(src, n, k, grp);
+  uint32_t umin = 0xFFFFFFFFu;
+  const int kept = group_emit<1>(src, n, sel, grp, [&](int pos, uint64_t K) {
+    scr[pos] = make_uint2(composite_value(K), composite_index(K));
+    umin = min(umin, composite_value(K));
+  });
+  umin = __reduce_min_sync(0xFFFFFFFFu, umin);
+  __syncwarp();
+  for (int pos = lane; pos < kept; pos += 32) seg[pos] = scr[pos];
+  __syncwarp();
+  if (lane == 0) {
+    if (kept >= k && umin != 0xFFFFFFFFu) atomicMax(&st->theta, umin + 1);
+    atomicAdd(stats + kStatCompactions, 1);
+  }
+  return kept;
+}
+
+// Raise a row's threshold to the lower edge of the histogram bin that holds
+// the k-th counted key (at least k keys of the row lie at or above it).  With
+// the key axis split over several units, the bound is shared through the
+// row's word in global memory: any unit's bound is a bound for the whole row.
+__device__ __forceinline__ void raise_theta(const uint32_t* h, RowState* st, int k, uint32_t* row_theta,
+                                         int lane) {
+  const Window w = window_of(ld_volatile_u64(&st->win));
+  uint32_t th = 0;
+  if (w.open) {
+    const Boundary B = find_boundary(h, static_cast<uint32_t>(k), lane);
+    if (B.found) {
+      const uint64_t t64 = static_cast<uint64_t>(w.base) + (static_cast<uint64_t>(B.bin) << w.shift);
+      th = t64 > 0xFFFFFFFFull ? 0xFFFFFFFFu : static_cast<uint32_t>(t64);
+    }
+  }
+  if (lane == 0) {
+    if (row_theta) th = max(th, atomicMax(row_theta, th));
+    if (th) atomicMax(&st->theta, th);
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 
 template <int R, bool PAGED, int MODE>
@@ -606,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       // chunks raised.
       for (int n = 0; ok; ++n) {
         const int qs = n & 3;
-        if (!wait_phase<true>(&uq_empty[qs], ((n >> 2) & 1) ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
+        if (!wait_phase<kSleep>(&uq_empty[qs], ((n >> 2) & 1) ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
         const int idx = atomicAdd(p.status + kSchedWord, 1);
         int u = -1;
         if (idx < p.num_units) {
@@ -619,16 +778,19 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         if (u < 0) break;
         const Unit U = get_unit<R, PAGED>(p, u);
         if (U.ntiles == 0) continue;
-        if (!wait_phase<true>(qempty, qphase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
+        if (!wait_phase<kProd>(qempty, qphase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
         qphase ^= 1;
         mbar_arrive_expect_tx(qfull, C::Q_BYTES);
         tma_load_2d(q_smem, &p.tmap_q, qfull, 0, U.row0 * kHeads);
         const int32_t* bt = PAGED ? p.block_table + static_cast<int64_t>(U.req) * p.max_blocks : nullptr;
         for (int t = 0; t < U.ntiles; ++t) {
-          if (!wait_phase<true>(&empty[stage], phase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
+          if (!wait_phase<kProd>(&empty[stage], phase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
           const int j0 = U.jbeg + t * kBlockKeys;
           uint8_t* dst = stage_smem + stage * C::TILE_BYTES;
-          if (!PAGED) {
+          if (p.debug_withhold_first_tile && n == 0 && t == 0) {
+            // tests only: this stage never fills, so the MMA's bounded wait on
+            // it runs out and the kernel takes its timeout path
+          } else if (!PAGED) {
             mbar_arrive_expect_tx(&full[stage], C::TILE_BYTES);
             tma_load_2d(dst, &p.tmap_k, &full[stage], 0, j0);
           } else {
@@ -643,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
             if (v0) tma_load_2d(dst, &p.tmap_k, &full[stage], 0, pg0 * kPageSize);
             if (v1) tma_load_2d(dst + 8192, &p.tmap_k, &full[stage], 0, pg1 * kPageSize);
           }
-          issued[stage] = true;
+          issued[stage] = !(p.debug_withhold_first_tile && n == 0 && t == 0);
           issued_phase[stage] = phase;
           if (++stage == S) {
             stage = 0;
@@ -671,21 +833,21 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       const uint32_t q_addr = smem_u32(q_smem);
       for (int n = 0; ok; ++n) {
         const int qs = n & 3;
-        if (!wait_phase<false>(&uq_full[qs], (n >> 2) & 1, abort_flag, p.status, limit)) { ok = false; break; }
+        if (!wait_phase<kSpin>(&uq_full[qs], (n >> 2) & 1, abort_flag, p.status, limit)) { ok = false; break; }
         const int u = uq[qs];
         mbar_arrive(&uq_empty[qs]);
         if (u < 0) break;
         const Unit U = get_unit<R, PAGED>(p, u);
         if (U.ntiles == 0) continue;
-        if (!wait_phase<false>(qfull, qphase, abort_flag, p.status, limit)) { ok = false; break; }
+        if (!wait_phase<kNap>(qfull, qphase, abort_flag, p.status, limit)) { ok = false; break; }
         qphase ^= 1;
         tc_fence_after();
         const uint64_t bdesc = smem_desc_k128_sw128(q_addr);
         for (int t = 0; t < U.ntiles; ++t, ++T) {
           const uint32_t a = T & 1, aph = (T >> 1) & 1;
-          if (!wait_phase<false>(&tempty[a], aph ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
+          if (!wait_phase<kNap>(&tempty[a], aph ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
           tc_fence_after();
-          if (!wait_phase<false>(&full[stage], phase, abort_flag, p.status, limit)) { ok = false; break; }
+          if (!wait_phase<kNap>(&full[stage], phase, abort_flag, p.status, limit)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = smem_desc_k128_sw128(smem_u32(stage_smem + stage * C::TILE_BYTES));
           const uint32_t d = tbase + a * N;
@@ -728,9 +890,9 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
 
     for (int it = 0;; ++it) {
       const int qs = it & 3;
-      const bool got = wait_phase<false>(&uq_full[qs], (it >> 2) & 1, abort_flag, p.status, limit);
+      const bool got = wait_phase<kSpin>(&uq_full[qs], (it >> 2) & 1, abort_flag, p.status, limit);
       // every warp of the group must take the same branch below (named barriers)
-      if (bar_red_or(bar_id, 128, !got)) {
+      if (bar_red_or(bar_id, 128, !got || aborted || *abort_flag)) {
         aborted = true;
         break;
       }
@@ -750,7 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
             for (int back = 2; back >= 1; --back) {
               if (it < back) continue;
               const int hslot = (it - back) & 1;
-              if (!wait_phase<true>(&slot_full[hslot], ((it - back) >> 1) & 1, abort_flag, p.status, limit)) break;
+              if (!wait_phase<kSleep>(&slot_full[hslot], ((it - back) >> 1) & 1, abort_flag, p.status, limit)) break;
               const SlotMeta meta = smeta[hslot];
               for (;;) {
                 int rl = 0;
@@ -765,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
             }
           }
           // tell the select group (unit -1 in the slot)
-          wait_phase<true>(&slot_empty[slot], ((it >> 1) & 1) ^ 1, abort_flag, p.status, limit);
+          wait_phase<kSleep>(&slot_empty[slot], ((it >> 1) & 1) ^ 1, abort_flag, p.status, limit);
           if (g == 0 && tid_wg == 0) smeta[slot].unit = -1;
           named_bar_sync(bar_id, 128);
           __syncwarp();
@@ -780,7 +942,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
                           ? p.cand + (static_cast<size_t>(blockIdx.x * 2 + slot) * R + g * RW) * cap
                           : nullptr;
       if (MODE == kModeTopK) {
-        if (!wait_phase<true>(&slot_empty[slot], ((it >> 1) & 1) ^ 1, abort_flag, p.status, limit)) aborted = true;
+        if (!wait_phase<kNap>(&slot_empty[slot], ((it >> 1) & 1) ^ 1, abort_flag, p.status, limit)) aborted = true;
       }
       // ---- per-row setup for this warpgroup's rows: the key range [lo, hi)
       // (kept in shared memory; the tile loop reads it back as a broadcast)
@@ -812,12 +974,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
           RowState& st = rs[tid_wg];
           st.wcnt[0] = st.wcnt[1] = st.wcnt[2] = st.wcnt[3] = 0;
           st.theta = 0;
-          st.theta_f = -INFINITY;
-          st.base = 0;
-          st.shift = 0;
-          st.mode = 0;
-          st.tmin = 0xFFFFFFFFu;
-          st.tmax = 0;
+          st.win = 0ull;
         }
         for (int x = tid_wg; x < RW * kNB; x += 128) hs[x] = 0;
         if (g == 0 && tid_wg == 0) {
@@ -846,22 +1003,25 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         }
       }
 
-      // ---- this warp's segment counts (reloaded after maintenance), its segment
-      // of each row's buffer, and the row state it reads once per vote period
-      int wcnt[RW];
-      uint2* seg[RW];
-      int lo[RW], span[RW], mode[RW], shift[RW];
-      uint32_t base[RW];
+      // ---- this warp's registers per row: candidates in its segment, how many of
+      // them the row's histogram has counted, the key range, and the threshold
+      // (reloaded from the row state at every vote)
+      // and the row's histogram window as this warp knows it (hbase = ~0 while
+      // closed: no key counts)
+      int cnt[RW], folded[RW], lo[RW], span[RW], hshift[RW];
+      uint32_t hbase[RW];
+      float thf[RW];
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
-        wcnt[r] = 0;
-        seg[r] = MODE == kModeTopK ? cand_s + static_cast<size_t>(r) * cap + qd * wcap : nullptr;
+        cnt[r] = 0;
+        folded[r] = 0;
         lo[r] = rs[r].lo;
         span[r] = rs[r].hi - rs[r].lo;
-        mode[r] = 0;
-        shift[r] = 0;
-        base[r] = 0;
+        thf[r] = -INFINITY;
+        hbase[r] = 0xFFFFFFFFu;
+        hshift[r] = 0;
       }
+      uint2* seg0 = MODE == kModeTopK ? cand_s + qd * wcap : nullptr;  // row r's segment: seg0 + r * cap
 
       // ---- stream the unit's key tiles
       const int key0 = U.jbeg + qd * 32 + lane;
@@ -873,13 +1033,13 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         return __ldg(p.s + static_cast<int64_t>(pg) * kPageSize + (j % kPageSize));
       };
       float s_next = U.ntiles ? scale_of(key0) : 0.f;
-      int next_vote = vote_interval(0) - 1;  // the same tile sequence in every warp of the group
+      int next_vote = vote_interval(0) - 1;  // the same tile sequence in every warp
       for (int t = 0; t < U.ntiles; ++t, ++T) {
         const int j = key0 + t * kBlockKeys;
         const float sj = 0.5f * s_next;  // relu_dot32_x2 returns twice the head sum
-        if (t + 1 < U.ntiles) s_next = scale_of(j + kBlockKeys);
+        s_next = scale_of(j + kBlockKeys);  // (0 past the end)
         const uint32_t a = T & 1, aph = (T >> 1) & 1;
-        if (!wait_phase<false>(&tfull[a], aph, abort_flag, p.status, limit)) aborted = true;
+        if (!wait_phase<kSpin>(&tfull[a], aph, abort_flag, p.status, limit)) aborted = true;
         tc_fence_after();
         float L[RW];
 #pragma unroll
@@ -891,10 +1051,11 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
           if (r + 2 == RW) {  // the accumulator is in registers now
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[a]);
+            mbar_arrive_if(lane == 0, &tempty[a]);
           }
-          L[r] = relu_dot32_x2(x0, ws_g + r * kHeads) * sj;
-          L[r + 1] = relu_dot32_x2(x1, ws_g + (r + 1) * kHeads) * sj;
+          // fma with +0: an exactly zero head sum gives +0 whatever the sign of the scale
+          L[r] = fmaf(relu_dot32_x2(x0, ws_g + r * kHeads), sj, 0.f);
+          L[r + 1] = fmaf(relu_dot32_x2(x1, ws_g + (r + 1) * kHeads), sj, 0.f);
         }
 
         if (MODE == kModeLogits) {
@@ -902,172 +1063,82 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
           for (int r = 0; r < RW; ++r) {
             if (g * RW + r >= U.nrows || j >= U.cend) continue;
             float* lrow = p.logits + static_cast<int64_t>(U.row0 + g * RW + r) * p.ld_logits;
-            __stcs(lrow + j, (j >= rs[r].lo && j < rs[r].hi) ? L[r] : -INFINITY);
+            __stcs(lrow + j, static_cast<uint32_t>(j - lo[r]) < static_cast<uint32_t>(span[r]) ? L[r] : -INFINITY);
           }
-          if (bar_red_or(bar_id, 128, aborted || *abort_flag)) {
-            aborted = true;
-            break;
-          }
+          if (aborted) break;
         } else {
-          // ---- filter against the running threshold; append to this warp's segment
-          float thf[RW];
-#pragma unroll
-          for (int r = 0; r < RW; ++r) thf[r] = rs[r].theta_f;  // may have risen last tile
+          // ---- filter against the row's threshold; append to this warp's segment
+          // and count the key into the row's histogram (once its window is open)
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
             const bool ps = static_cast<uint32_t>(j - lo[r]) < static_cast<uint32_t>(span[r]) && L[r] >= thf[r];
             const uint32_t msk = __ballot_sync(0xFFFFFFFFu, ps);
-            const uint32_t key = order_key(L[r]);
-            const int pos = wcnt[r] + __popc(msk & lt);
-            wcnt[r] += __popc(msk);
-            st_global_v2_if(ps && pos < wcap, seg[r] + pos, key, static_cast<uint32_t>(j));
-            const int hidx = r * kNB + hist_index(hist_bin(key, base[r], shift[r]));
-            red_shared_add_if(ps && mode[r] == 1 && key >= base[r], hs + hidx, 1u);
+            const int pos = cnt[r] + __popc(msk & lt);
+            cnt[r] += __popc(msk);
+            const uint32_t key = order_key_nz(L[r]);
+            st_global_v2_if(ps && pos < wcap, seg0 + static_cast<size_t>(r) * cap + pos, key,
+                            static_cast<uint32_t>(j));
+            red_shared_add_if(ps && key >= hbase[r], hs + r * kNB + hist_bin(key, hbase[r], hshift[r]), 1u);
           }
-          // At every vote tile (and the last), one barrier carries two votes:
-          // abort (weight 1: lane 0 of each warp) and maintenance (weight 5:
-          // lanes 0..4 of each warp): a row still without its histogram window
-          // has candidates, or a segment is within 32 * kMaxVoteTiles of full.
+          // ---- vote: count, make room, reload the thresholds (this warp alone)
           if (t == next_vote || t + 1 == U.ntiles) {
-            next_vote = t + vote_interval(t + 1);
-            bool maint = false;
-#pragma unroll
-            for (int r = 0; r < RW; ++r) {
-              maint |= (mode[r] == 0 && wcnt[r] > 0) || wcnt[r] > wcap - kMaxVoteTiles * 32;
-              if (wcnt[r] > wcap && lane == 0) atomicOr(p.status, kStatusCandOverflow);
-            }
-            if (lane == 0) {
-#pragma unroll
-              for (int r = 0; r < RW; ++r) rs[r].wcnt[qd] = min(wcnt[r], wcap);
-            }
-            const bool ab = aborted || *abort_flag;
-            const uint32_t votes = bar_red_popc(bar_id, 128, (lane == 0 && ab) || (lane < 5 && maint));
-            if (votes % 5) {
+            const int vnext = vote_interval(t + 1);
+            next_vote = t + vnext;
+            if (aborted || *abort_flag) {
               aborted = true;
               break;
             }
-            if (votes >= 5) {
-              // Quiescent point: every warp of the group is here.  Snapshot, then act.
-              bool opened[RW], compact[RW];
+            const int room = min(vnext, U.ntiles - 1 - t) * 32;  // what may be appended before the next vote
+            bool full = false;
 #pragma unroll
-              for (int r = 0; r < RW; ++r) {
-                const RowState& st = rs[r];
-                opened[r] = st.mode == 0 && (st.wcnt[0] + st.wcnt[1] + st.wcnt[2] + st.wcnt[3]) > 0;
-                compact[r] = max(max(st.wcnt[0], st.wcnt[1]), max(st.wcnt[2], st.wcnt[3])) > wcap - kMaxVoteTiles * 32;
+            for (int r = 0; r < RW; ++r) {
+              if (cnt[r] > wcap && lane == 0) atomicOr(p.status, kStatusCandOverflow);
+              cnt[r] = min(cnt[r], wcap);
+              if (hbase[r] == 0xFFFFFFFFu && cnt[r] > 0) {
+                // once per row: open the window (or take the one another warp
+                // opened) and count what was appended before it
+                folded[r] = fold_segment(seg0 + static_cast<size_t>(r) * cap, folded[r], cnt[r], rs + r,
+                                         hs + r * kNB, lane);
+                const Window w = window_of(ld_volatile_u64(&rs[r].win));
+                hbase[r] = w.base;
+                hshift[r] = w.shift;
               }
-              named_bar_sync(bar_id, 128);
-              if (qd < RW && (compact[qd] || opened[qd])) {
-                RowState& st = rs[qd];
-                uint2* rowbuf = cand_s + static_cast<size_t>(qd) * cap;
-                uint32_t* h = hs + qd * kNB;
-                if (opened[qd]) {
-                  // Open the row's histogram window over twice the span of the keys
-                  // collected so far (at most kMaxVoteTiles tiles' worth) and count them.
-                  uint32_t kmin = 0xFFFFFFFFu, kmax = 0;
-                  for (int s = 0; s < 4; ++s)
-                    for (int e = lane; e < st.wcnt[s]; e += 32) {
-                      const uint32_t key = rowbuf[s * wcap + e].x;
-                      kmin = min(kmin, key);
-                      kmax = max(kmax, key);
-                    }
-                  kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
-                  kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
-                  const uint64_t span = static_cast<uint64_t>(kmax - kmin);
-                  const int bits = 64 - __clzll(static_cast<long long>(2 * span + 1));
-                  const uint32_t wbase = kmin;
-                  const int wshift = bits > 9 ? bits - 9 : 0;
-                  if (!compact[qd])
-                    for (int s = 0; s < 4; ++s)
-                      for (int e = lane; e < st.wcnt[s]; e += 32) {
-                        const uint32_t key = rowbuf[s * wcap + e].x;
-                        atomicAdd(&h[hist_index(hist_bin(key, wbase, wshift))], 1u);
-                      }
-                  __syncwarp();
-                  if (lane == 0) {
-                    st.base = wbase;
-                    st.shift = wshift;
-                    st.mode = 1;
-                  }
-                  __syncwarp();
-                }
-                if (compact[qd]) {
-                  // Rare: a segment is near full.  Keep the row's exact top-k (later keys
-                  // have larger indices, so a key equal to the k-th value never enters
-                  // again), staged through scratch and dealt back over the segments.
-                  const SegSrc src{rowbuf, wcap, st.wcnt[0], st.wcnt[1], st.wcnt[2], st.wcnt[3]};
-                  uint2* scr = p.scratch + (static_cast<size_t>(blockIdx.x) * 8 + ew) * k;
-                  const SelectResult sel = group_select<1>(src, 4 * wcap, k, grp);
-                  uint32_t umin = 0xFFFFFFFFu;
-                  const int kept = group_emit<1>(src, 4 * wcap, sel, grp, [&](int pos, uint64_t K) {
-                    scr[pos] = make_uint2(composite_value(K), composite_index(K));
-                    umin = min(umin, composite_value(K));
-                  });
-                  umin = __reduce_min_sync(0xFFFFFFFFu, umin);
-                  __syncwarp();
-                  for (int pos = lane; pos < kept; pos += 32) rowbuf[(pos & 3) * wcap + (pos >> 2)] = scr[pos];
-                  if (lane == 0) {
-                    for (int s = 0; s < 4; ++s) st.wcnt[s] = (kept - s + 3) / 4;
-                    if (kept >= k) {
-                      st.theta = max(st.theta, umin == 0xFFFFFFFFu ? umin : umin + 1);
-                      st.theta_f = theta_float(st.theta);
-                    }
-                    atomicAdd(p.status + kStatCompactions, 1);
-                  }
-                  for (int x = lane; x < kNB; x += 32) h[x] = 0;
-                  __syncwarp();
-                  for (int e = lane; e < kept; e += 32) {
-                    const uint32_t key = scr[e].x;
-                    if (key >= st.base) atomicAdd(&h[hist_index(hist_bin(key, st.base, st.shift))], 1u);
-                  }
-                }
-              }
-              named_bar_sync(bar_id, 128);
+              folded[r] = cnt[r];  // the hot loop counts from here on
+              full |= cnt[r] + room > wcap;
+            }
+            while (full) {  // rare: one row at a time, through a single copy of the compaction
+              int cr = -1, cc = 0;
 #pragma unroll
-              for (int r = 0; r < RW; ++r) wcnt[r] = rs[r].wcnt[qd];
-            }
+              for (int r = RW - 1; r >= 0; --r)
+                if (cnt[r] + room > wcap) {
+                  cr = r;
+                  cc = cnt[r];
+                }
+              if (cr < 0) break;
+              uint2* scr = p.scratch + (static_cast<size_t>(blockIdx.x) * 8 + ew) * k;
+              const int nc = compact_segment(seg0 + static_cast<size_t>(cr) * cap, cc, room, wcap, k, rs + cr, scr,
+                                             grp, p.status, lane);
 #pragma unroll
-            for (int r = 0; r < RW; ++r) {  // histogram windows may have opened
-              mode[r] = rs[r].mode;
-              base[r] = rs[r].base;
-              shift[r] = rs[r].shift;
+              for (int r = 0; r < RW; ++r)
+                if (r == cr) cnt[r] = folded[r] = nc;
             }
-            // ---- raise the threshold from the histogram (warp qd for row qd).  With the
-            // key axis split over several units, the row's bound is shared through
-            // global memory: any unit's histogram bound (at least k keys of the row
-            // lie at or above it) is a bound for the whole row.
-            if (qd < RW && g * RW + qd < U.nrows) {
-              RowState& st = rs[qd];
-              uint32_t th = 0;
-              if (mode[qd] == 1) {
-                const Boundary B = find_boundary(hs + qd * kNB, static_cast<uint32_t>(k), lane);
-                if (B.found) {
-                  const uint64_t t64 = static_cast<uint64_t>(st.base) + (static_cast<uint64_t>(B.bin) << st.shift);
-                  th = t64 > 0xFFFFFFFFull ? 0xFFFFFFFFu : static_cast<uint32_t>(t64);
-                }
-              }
-              if (lane == 0) {
-                if (p.n_chunks > 1) {
-                  const uint32_t gbound = atomicMax(p.row_theta + U.row0 + g * RW + qd, th);
-                  th = max(th, gbound);
-                }
-                if (th > st.theta) {
-                  st.theta = th;
-                  st.theta_f = theta_float(th);
-                }
-              }
-            }
+            if (qd < RW && g * RW + qd < U.nrows)
+              raise_theta(hs + qd * kNB, rs + qd, k, p.n_chunks > 1 ? p.row_theta + U.row0 + g * RW + qd : nullptr,
+                          lane);
+#pragma unroll
+            for (int r = 0; r < RW; ++r) thf[r] = theta_float(ld_volatile_u32(&rs[r].theta));
           }
         }
       }
-      if (aborted) break;
+      // (an aborted warp carries on to the next unit's group vote, which ends
+      // the loop for every warp of the group together)
       if (MODE == kModeTopK) {
         if (lane == 0) {
 #pragma unroll
-          for (int r = 0; r < RW; ++r) rs[r].wcnt[qd] = min(wcnt[r], wcap);
+          for (int r = 0; r < RW; ++r) rs[r].wcnt[qd] = cnt[r];
         }
-        named_bar_sync(bar_id, 128);  // every warp's row-state writes are done
         __syncwarp();
-        if (lane == 0) mbar_arrive(&slot_full[slot]);
+        if (lane == 0) mbar_arrive(&slot_full[slot]);  // releases this warp's row-state and candidate writes
       }
     }
   } else if (MODE == kModeTopK) {
@@ -1080,7 +1151,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
     const int wcap = cap >> 2;
     for (int it = 0;; ++it) {
       const int slot = it & 1;
-      const bool ok = wait_phase<true>(&slot_full[slot], (it >> 1) & 1, abort_flag, p.status, limit);
+      const bool ok = wait_phase<kSleep>(&slot_full[slot], (it >> 1) & 1, abort_flag, p.status, limit);
       if (bar_red_or(kSelBar, NT, !ok || *abort_flag)) break;
       const SlotMeta meta = smeta[slot];
       if (meta.unit < 0) break;
@@ -1135,7 +1206,7 @@ struct PartSrc {
   __device__ __forceinline__ bool get(int e, uint64_t& K) const {
     const int c = e / topk;
     const int i = e - c * topk;
-    if (i >= __ldg(cnt + static_cast<size_t>(c) * cstride)) return false;
+    if (i >= __ldg(cnt + static_cast<size_t>(c) * cstride)) return false;  // (i < topk always)
     const uint2 v = base[static_cast<size_t>(c) * stride + i];
     K = compose_key(v.x, v.y);
     return true;
@@ -1178,7 +1249,9 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
   int total = -1;  // pairs surviving in all chunks (-1: not scanned)
   if (p.n_chunks <= kMergeMaxChunks) {
     const int c = threadIdx.x;
-    const int v = c < p.n_chunks ? __ldg(cnt + static_cast<size_t>(c) * p.R) : 0;
+    // a count outside [0, topk] only follows an aborted indexer launch (the
+    // device status says so); clamped, it still keeps every access in bounds
+    const int v = c < p.n_chunks ? min(max(__ldg(cnt + static_cast<size_t>(c) * p.R), 0), p.topk) : 0;
     int incl = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {

@@ -70,6 +70,7 @@ struct IndexerParams {
   int* part_cnt;    // split mode: [num_units][R]
   uint32_t* row_theta;  // split mode: [m] best lower bound on each row's k-th order key, zeroed per call
   unsigned long long wait_limit_ns;
+  int debug_withhold_first_tile;  // tests only: never issue the first key tile's load (its wait runs out)
 };
 
 struct MergeParams {

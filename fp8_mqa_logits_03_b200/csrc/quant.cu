@@ -6,7 +6,8 @@
 //   s_t   = max(max_d |x[t,d]|, 1e-4) / 448            (fp32)
 //   q_t,d = e4m3(x[t,d] / s_t), nearest even, saturating at +-448
 // and the codes and the scale go to pool slot slot[t] (page slot / 64, row
-// slot % 64).  A slot outside [0, num_slots) is not stored.
+// slot % 64).  A slot outside [0, num_slots) is not stored.  NaN elements
+// are left out of the row maximum and get a NaN code (0x7F or 0xFF).
 //
 // One warp per 4 tokens: each lane first loads 4 bf16 (8 bytes) of each of
 // the 4 rows, so that a warp has 1 KB in flight (the rows are read in
@@ -31,6 +32,11 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_sat(float lo, float hi) {
   return r;
 }
 
+__device__ __forceinline__ uint32_t abs_bits_no_nan(float f) {
+  const uint32_t b = __float_as_uint(f) & 0x7FFFFFFFu;
+  return b > 0x7F800000u ? 0u : b;
+}
+
 __global__ void __launch_bounds__(kQuantWarps * 32)
     act_quant_store_kernel(const uint16_t* __restrict__ x, int64_t T, const int64_t* __restrict__ slot,
                            int64_t num_slots, uint8_t* __restrict__ k_pool, float* __restrict__ s_pool) {
@@ -49,9 +55,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
     if (sl[i] < 0 || sl[i] >= num_slots) continue;  // the same for the whole warp
     const float f0 = __uint_as_float(raw[i].x << 16), f1 = __uint_as_float(raw[i].x & 0xFFFF0000u);
     const float f2 = __uint_as_float(raw[i].y << 16), f3 = __uint_as_float(raw[i].y & 0xFFFF0000u);
-    // |x| as bits: non-negative floats order like their bit patterns
-    uint32_t a = max(max(__float_as_uint(fabsf(f0)), __float_as_uint(fabsf(f1))),
-                     max(__float_as_uint(fabsf(f2)), __float_as_uint(fabsf(f3))));
+    // |x| as bits: non-negative floats order like their bit patterns; a NaN
+    // (bits above +inf's) counts as 0, so the row maximum is over the rest
+    uint32_t a = max(max(abs_bits_no_nan(f0), abs_bits_no_nan(f1)), max(abs_bits_no_nan(f2), abs_bits_no_nan(f3)));
     a = __reduce_max_sync(0xFFFFFFFFu, a);
     const float sc = fmaxf(__uint_as_float(a), 1e-4f) / 448.0f;
     const uint32_t lo = e4m3x2_rn_sat(f0 / sc, f1 / sc);

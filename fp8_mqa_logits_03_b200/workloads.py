@@ -63,7 +63,8 @@ def _fp8_bytes(x: torch.Tensor) -> torch.Tensor:
 
 
 def make_prefill(m: int, n: int, seed: int, rank_start: int | None = None, ks=None, ke=None,
-                 heads: int = H, dim: int = D, duplicate_keys: bool = False) -> dict:
+                 heads: int = H, dim: int = D, duplicate_keys: bool = False,
+                 signed_weights: bool = False) -> dict:
     """Ragged-prefill inputs as CPU tensors.
 
     q [m, heads, dim] uint8, k [n, dim] uint8, s [n] f32, w [m, heads] f32,
@@ -71,12 +72,15 @@ def make_prefill(m: int, n: int, seed: int, rank_start: int | None = None, ks=No
     clamped to n (rank_start defaults to n - m, a causal tail).  Explicit
     ks/ke override the defaults.  duplicate_keys=True makes every key the
     same vector with scale 1 (a degenerate all-ties case).
+    signed_weights=True draws w ~ U[-1, 1) instead of U[0, 1).
     """
     g = torch.Generator().manual_seed(seed)
     q = _fp8_bytes(torch.randn(m, heads, dim, generator=g))
     k = _fp8_bytes(torch.randn(n, dim, generator=g))
     s = torch.rand(n, generator=g) + 0.5
     w = torch.rand(m, heads, generator=g)
+    if signed_weights:
+        w = 2.0 * w - 1.0
     if duplicate_keys and n > 0:
         k = k[:1].expand(n, dim).contiguous()
         s = torch.ones(n)
@@ -93,7 +97,8 @@ def make_prefill(m: int, n: int, seed: int, rank_start: int | None = None, ks=No
 
 
 def make_paged(B: int, R: int, lmin: int, lmax: int, seed: int, page_size: int = PAGE_SIZE,
-               heads: int = H, dim: int = D, lengths=None, max_blocks: int | None = None) -> dict:
+               heads: int = H, dim: int = D, lengths=None, max_blocks: int | None = None,
+               signed_weights: bool = False) -> dict:
     """Paged-decode inputs as CPU tensors.
 
     Context lengths L_b ~ U{lmin..lmax} (both ends inclusive) unless given.
@@ -101,7 +106,8 @@ def make_paged(B: int, R: int, lmin: int, lmax: int, seed: int, page_size: int =
     one seeded random permutation.  block_table [B, max_blocks] int32 holds
     the physical page of each logical page, padded with -1.  k_pages
     [P, page_size, dim] uint8, s_pages [P, page_size] f32, q [B*R, heads,
-    dim] uint8, w [B*R, heads] f32, seq_lens [B] int32.
+    dim] uint8, w [B*R, heads] f32, seq_lens [B] int32.  signed_weights=True
+    draws w ~ U[-1, 1) instead of U[0, 1).
     """
     g = torch.Generator().manual_seed(seed)
     if lengths is None:
@@ -122,6 +128,8 @@ def make_paged(B: int, R: int, lmin: int, lmax: int, seed: int, page_size: int =
     k_pages = _fp8_bytes(torch.randn(max(P, 1), page_size, dim, generator=g))
     s_pages = torch.rand(max(P, 1), page_size, generator=g) + 0.5
     w = torch.rand(B * R, heads, generator=g)
+    if signed_weights:
+        w = 2.0 * w - 1.0
     return dict(q=q.contiguous(), k_pages=k_pages.contiguous(), s_pages=s_pages.contiguous(),
                 w=w.contiguous(), block_table=block_table.contiguous(),
                 seq_lens=lengths.to(torch.int32).contiguous(), B=B, R=R, P=P,

@@ -147,9 +147,14 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
  * Large problems run on fewer SMs so that the workspace fits; a problem that
  * does not fit at all returns FP8IDX_EWORKSPACE.  All calls share the array:
  * calls that can overlap on the GPU race and must be serialised by the
- * caller.  The device status of the last call is not readable through this
- * entry point's interface.
+ * caller.  The status block of the last call is the head of that array: read
+ * it with fp8idx_read_device_status(FP8IDX_NOALLOC_WS, ...) (and the stats
+ * likewise).  The array's device address is looked up once per device index
+ * and kept for the life of the process, so the library must not be used
+ * across a cudaDeviceReset (or any teardown of the primary context), after
+ * which the array may live elsewhere.
  */
+#define FP8IDX_NOALLOC_WS ((const void*)1)
 int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const float* s,
                                    const float* w, const int32_t* ks, const int32_t* ke, int64_t m,
                                    int64_t n, int H, int D, int topk, int32_t* out_idx,
@@ -169,6 +174,8 @@ int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const flo
  *   slot    [T] int64, 8-byte aligned
  *   k_pool  [num_slots, 128] e4m3 bytes (k_pages viewed as slots), 4-byte aligned
  *   s_pool  [num_slots] fp32 (s_pages viewed as slots), 4-byte aligned
+ * NaN elements of x are left out of the row maximum and get a NaN code
+ * (0x7F or 0xFF); the other codes of the row are unaffected.
  * Slots not named by any token are left untouched; two tokens naming one
  * slot race.  No workspace.
  */
@@ -176,9 +183,64 @@ int fp8idx_act_quant_store(const uint16_t* x, int64_t T, int D, const int64_t* s
                            uint8_t* k_pool, float* s_pool, void* stream);
 
 /*
+ * Index preparation (the `gen_nsa_ks_ke` step of the "reuse inference
+ * metadata and streamline FP8 prefill" page: its description table, the
+ * walkthrough of the ragged-index copy, and the review's expected ragged
+ * buffer).  B requests are laid out back to back in one ragged key space:
+ * request b owns key positions [koff_b, koff_b + seq_len[b]), koff_b the sum
+ * of the earlier seq_len; its query rows (its last q_len[b] tokens) are rows
+ * [qoff_b, qoff_b + q_len[b]) of the batch, qoff_b the sum of the earlier
+ * q_len.  For row t of request b:
+ *     ks = koff_b,  ke = koff_b + clamp(seq_len[b] - q_len[b] + t + 1, 0, seq_len[b]),
+ *     row_table = req_idx[b]                          (the row's token-table row),
+ * and, when `ragged` is not NULL, the token slots of every request are copied
+ * in the same order (the long-context copy, parallel over all positions):
+ *     ragged[koff_b + p] = req_to_token[req_idx[b] * ld_table + p],  p < seq_len[b]
+ * (-1 where req_idx[b] is outside [0, table_rows) or p >= ld_table).
+ *   seq_len, q_len, req_idx [B] int32 (negative lengths count as 0); B <= 8192
+ *   req_to_token  [table_rows, ld_table] int32 token slots (LightLLM's
+ *                 req_to_token_indexs; several requests may share a row, as
+ *                 the HOLD padding requests do)
+ *   ks, ke        [q_cap] int32; rows past the batch's sum of q_len are
+ *                 written empty (ks = ke = 0, row_table = -1)
+ *   row_table     [q_cap] int32 or NULL
+ *   ragged        [ragged_cap] int32 or NULL; positions past the batch's sum
+ *                 of seq_len are not written
+ * The sums are formed on the device, so the call never reads device data on
+ * the host: the caller sizes q_cap and ragged_cap as upper bounds, and every
+ * key position must stay below 2^31.  No workspace.
+ */
+int fp8idx_prepare_ragged(const int32_t* seq_len, const int32_t* q_len, const int32_t* req_idx, int B,
+                          const int32_t* req_to_token, int64_t table_rows, int64_t ld_table, int32_t* ks,
+                          int32_t* ke, int32_t* row_table, int64_t q_cap, int32_t* ragged, int64_t ragged_cap,
+                          void* stream);
+
+/*
+ * Top-k transform: selected key positions to physical slots through a page
+ * table (the `page_table_size_1` argument of `fast_topk_transform_fused`,
+ * "bench_mqa_logits_chunking.py" page; with page_size 64 the block table of
+ * the paged form).  For row i and each r < topk:
+ *     p = idx[i, r] - row_base[i]           (row_base NULL: 0)
+ *     t = row_table[i]                      (row_table NULL: i / rows_per_table_row)
+ *     out[i, r] = page_table[t * ld_table + p / page_size] * page_size + p % page_size
+ * and -1 where idx[i, r] is negative, p < 0, t is outside [0, table_rows),
+ * p / page_size >= ld_table, or the table entry is negative.  With the rows
+ * of fp8idx_prepare_ragged: row_base = ks, row_table = its row_table, the
+ * token table and page_size 1.  With the paged form's output: row_base NULL,
+ * rows_per_table_row = R, the block table and page_size 64.
+ *   idx, out [rows, topk] int32 (may be the same buffer); slots must fit int32.
+ * No workspace.
+ */
+int fp8idx_topk_transform(const int32_t* idx, int64_t rows, int topk, const int32_t* row_base,
+                          const int32_t* row_table, int rows_per_table_row, const int32_t* page_table,
+                          int64_t table_rows, int64_t ld_table, int page_size, int32_t* out, void* stream);
+
+/*
  * Tests and diagnostics.  fp8idx_read_device_status synchronises `stream`
  * and copies the status word written by the last call that used workspace
- * `ws` (ws == NULL: the last fp8idx_mqa_logits call) into *status_out.
+ * `ws` into *status_out.  ws == NULL names the last fp8idx_mqa_logits call,
+ * ws == FP8IDX_NOALLOC_WS the last fp8idx_mqa_logits_topk_noalloc call on
+ * the current device.
  */
 int fp8idx_read_device_status(const void* ws, int* status_out, void* stream);
 /* Copies the first `count` (<= 64) 32-bit words of a workspace's status block:
@@ -193,8 +255,17 @@ const char* fp8idx_last_error(void);
 /* Number of SMs of the current device (what the workspace sizes assume). */
 int fp8idx_num_sms(void);
 /* Upper bound in nanoseconds on any single pipeline wait inside a kernel
- * (default 2e9).  Tests lower it to exercise the timeout path. */
+ * (default 2e9), taken by calls made after it.  With 0, every wait that does
+ * not succeed at once gives up: the kernel sets FP8IDX_STATUS_WAIT_TIMEOUT,
+ * drains its own copies and returns (the tests use this to exercise the
+ * timeout path). */
 void fp8idx_set_wait_limit_ns(uint64_t ns);
+/* Tests only (no counterpart on the pages).  While `on` is nonzero, each CTA
+ * of the fused and paged calls made afterwards never issues the load of its
+ * first key tile, so the MMA's bounded wait on that tile runs out after the
+ * wait limit: the call returns with FP8IDX_STATUS_WAIT_TIMEOUT set and its
+ * outputs invalid, and the context stays usable.  Off by default. */
+void fp8idx_debug_withhold_first_tile(int on);
 
 #ifdef __cplusplus
 }

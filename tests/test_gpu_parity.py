@@ -126,6 +126,26 @@ def test_fused_small(m, n, k, seed):
     _check_fused(d, idx.cpu().numpy(), vals.cpu().numpy(), np.arange(m), k)
 
 
+@pytest.mark.parametrize("m,n,k,seed", [(13, 9000, 2048, 41), (8 * 148 + 3, 5000, 512, 42)])
+def test_fused_signed_weights(m, n, k, seed):
+    """Head weights of both signs, w ~ U[-1, 1): heads cancel in the weighted sum,
+    which is where the epilogue's w*x + w*|x| form and the plain ReLU form differ most."""
+    ks, ke = _ragged(m, n, seed)
+    d = workloads.make_prefill(m, n, seed, ks=ks, ke=ke, signed_weights=True)
+    idx, vals = _fused_call(d, k)
+    rows = np.arange(m) if m < 64 else np.concatenate([np.arange(0, 16), np.arange(m - 16, m)])
+    _check_fused(d, idx.cpu().numpy(), vals.cpu().numpy(), rows, k)
+
+
+def test_mqa_logits_signed_weights():
+    m, n = 24, 3000
+    ks, ke = _ragged(m, n, 43)
+    d = workloads.make_prefill(m, n, 43, ks=ks, ke=ke, signed_weights=True)
+    lg = fx.mqa_logits(**_to(d))
+    torch.cuda.synchronize()
+    check_logits(lg.cpu().numpy(), _oracle_rows(d, np.arange(m)))
+
+
 @pytest.mark.parametrize("k", [2048, 100])
 def test_fused_unsplit_schedule(k):
     """>= 8 x SMs rows: one unit per row block, top-k written directly."""
@@ -194,6 +214,16 @@ def test_paged_small(R, k):
     idx, vals = fx.paged_mqa_logits_topk(**t, R=R, topk=k, return_values=True, workspace=ws)
     assert fx.read_device_status(ws) == 0
     _paged_check(d, idx.cpu().numpy(), vals.cpu().numpy(), np.arange(len(lengths) * R), k)
+
+
+def test_paged_signed_weights():
+    lengths = [5000, 300, 4200, 64, 2049, 9000]
+    d = workloads.make_paged(len(lengths), 4, 1, 9000, seed=44, lengths=lengths, signed_weights=True)
+    t = {key: d[key].cuda() for key in ("q", "k_pages", "s_pages", "w", "block_table", "seq_lens")}
+    ws = fx.alloc_workspace(fx.paged_workspace_size(len(lengths), 4, d["max_blocks"], 2048))
+    idx, vals = fx.paged_mqa_logits_topk(**t, R=4, topk=2048, return_values=True, workspace=ws)
+    assert fx.read_device_status(ws) == 0
+    _paged_check(d, idx.cpu().numpy(), vals.cpu().numpy(), np.arange(len(lengths) * 4), 2048)
 
 
 # ---------------------------------------------------------------------------- full sizes (sampled)

@@ -7,7 +7,9 @@ library exposes fp8idx_mqa_logits_topk_noalloc, which takes its scratch from a
 fixed device array inside the library instead of a caller workspace.  This
 file calls it through the C ABI twice in a row (the array keeps the previous
 call's contents) and checks each result against fp8idx_mqa_logits_topk on the
-same inputs.  It is collected last so that a run stopping at the first failure
+same inputs, reading the call's device status through the same ABI
+(FP8IDX_NOALLOC_WS); one shape is also checked against the float64 oracle
+directly.  It is collected last so that a run stopping at the first failure
 has already run every other test.
 """
 import ctypes
@@ -16,8 +18,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import fp8_mqa_logits_03_b200 as fx
 from fp8_mqa_logits_03_b200 import workloads
+from _parity import check_topk_row, row_range
 
 pytestmark = pytest.mark.gpu
 
@@ -37,6 +41,15 @@ def L():
                                                    vp, vp, vp]
     lib.fp8idx_mqa_logits_topk_noalloc.restype = ctypes.c_int
     return lib
+
+
+NOALLOC_WS = ctypes.c_void_p(1)  # FP8IDX_NOALLOC_WS
+
+
+def _noalloc_status(L, stream):
+    v = ctypes.c_int(-1)
+    assert L.fp8idx_read_device_status(NOALLOC_WS, ctypes.byref(v), stream) == 0, L.fp8idx_last_error()
+    return v.value
 
 
 def _p(t):
@@ -79,11 +92,33 @@ def test_noalloc_matches_workspace_entry_point_twice(L, m, n, k, seed):
                                               _p(t["ks"]), _p(t["ke"]), m, n, 32, 128, k, _p(out),
                                               _p(vals), stream)
         assert rc == 0, L.fp8idx_last_error()
-        torch.cuda.synchronize()
+        assert _noalloc_status(L, stream) == 0
         oi, ov = out.cpu().numpy(), vals.cpu().numpy()
         rows = range(m) if m <= 1200 else np.linspace(0, m - 1, 200).astype(int)
         for i in rows:
             _same_topk(oi[i], ov[i], ref_i[i], ref_v[i], k, f"call {call} row {i}")
+
+
+def test_noalloc_matches_oracle(L):
+    m, n, k = 24, 5000, 512
+    g = np.random.default_rng(12)
+    ks = g.integers(0, 200, size=m).astype(np.int32)
+    ke = (ks + g.integers(100, n, size=m)).astype(np.int32)
+    d = workloads.make_prefill(m, n, 12, ks=ks, ke=ke)
+    t = {x: d[x].cuda() for x in ("q", "k", "s", "w", "ks", "ke")}
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    out = torch.empty((m, k), dtype=torch.int32, device="cuda")
+    vals = torch.empty((m, k), dtype=torch.float32, device="cuda")
+    rc = L.fp8idx_mqa_logits_topk_noalloc(_p(t["q"]), _p(t["k"]), _p(t["s"]), _p(t["w"]), _p(t["ks"]),
+                                          _p(t["ke"]), m, n, 32, 128, k, _p(out), _p(vals), stream)
+    assert rc == 0, L.fp8idx_last_error()
+    assert _noalloc_status(L, stream) == 0
+    ref = oracle.mqa_logits_rows(d["q"].numpy(), d["k"].numpy(), d["s"].numpy(), d["w"].numpy(),
+                                 d["ks"].numpy(), d["ke"].numpy(), rows=np.arange(m))
+    oi, ov = out.cpu().numpy(), vals.cpu().numpy()
+    for i in range(m):
+        lo, hi = row_range(d["ks"][i], d["ke"][i], n)
+        check_topk_row(oi[i], ref[i], lo, hi, k, ov[i], f"row {i}")
 
 
 def test_noalloc_rejects_bad_arguments(L):
