@@ -151,10 +151,10 @@ def read_device_status(workspace=None, stream=None) -> int:
 
 def read_device_stats(workspace, stream=None) -> dict:
     """Counters the fused top-k left in a workspace's status block (tuning aid)."""
-    buf = (ctypes.c_uint32 * 5)()
-    _check(lib().fp8idx_read_device_stats(_ws_ptr(workspace), buf, 5, _stream(stream)))
+    buf = (ctypes.c_uint32 * 6)()
+    _check(lib().fp8idx_read_device_stats(_ws_ptr(workspace), buf, 6, _stream(stream)))
     return dict(status=buf[0], compactions=buf[1], general_selects=buf[2], candidates=buf[3],
-                max_boundary=buf[4])
+                max_boundary=buf[4], repairs=buf[5])
 
 
 # ---------------------------------------------------------------------------- calls

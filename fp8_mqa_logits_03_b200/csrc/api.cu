@@ -122,9 +122,14 @@ struct Plan {
   int n_chunks = 1;
   int chunk_keys = 0;
   int num_units = 0;
+  int groups = 0;      // row blocks (prefill) or requests (paged)
+  int64_t axis = 0;    // the whole key axis
   int grid = 0;
   int cap = 0;
-  size_t off_cand = 0, off_scratch = 0, off_part = 0, off_cnt = 0, off_theta = 0, total = 0;
+  int rgrid = 0;       // CTAs of the repair launch
+  int rcap = 0;        // its candidate capacity per row (whole rows)
+  size_t off_cand = 0, off_scratch = 0, off_part = 0, off_cnt = 0, off_theta = 0, off_spec = 0,
+         off_repair = 0, off_rcand = 0, total = 0;
 };
 
 // Room for the candidates a row collects over `keys` keys (four equal
@@ -145,6 +150,8 @@ int candidate_capacity(int topk, int64_t keys) {
 }
 
 void finish_plan(Plan& pl, int64_t groups, int sms, int topk, int64_t axis) {
+  pl.groups = static_cast<int>(groups);
+  pl.axis = axis;
   pl.num_units = static_cast<int>(groups * pl.n_chunks);
   pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(pl.num_units, sms)));
   pl.cap = candidate_capacity(topk, std::min<int64_t>(axis, pl.chunk_keys));
@@ -153,23 +160,94 @@ void finish_plan(Plan& pl, int64_t groups, int sms, int topk, int64_t axis) {
   // two row-state slots per CTA (a unit is selected while the next one streams)
   off += round_up(static_cast<int64_t>(2) * sms * pl.R * pl.cap * 8, 256);
   pl.off_scratch = off;  // staging for a rare in-kernel compaction, per epilogue warp
-  off += round_up(static_cast<int64_t>(sms) * 8 * topk * 8, 256);
+  off += round_up(static_cast<int64_t>(sms) * kMaxEpiWarps * topk * 8, 256);
+  pl.off_repair = off;   // per group: listed flag, then the list
+  off += round_up(groups * 2 * 4, 256);
+  pl.rgrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({groups, sms, kRepairMaxGrid})));
   if (pl.n_chunks > 1) {
     pl.off_part = off;
     off += round_up(static_cast<int64_t>(pl.num_units) * pl.R * topk * 8, 256);
     pl.off_cnt = off;
     off += round_up(static_cast<int64_t>(pl.num_units) * pl.R * 4, 256);
-    pl.off_theta = off;  // per-row shared threshold
+    pl.off_theta = off;  // per-row shared threshold, then per-row largest estimate
     off += round_up(groups * pl.R * 4, 256);
+    pl.off_spec = off;
+    off += round_up(groups * pl.R * 4, 256);
+    // a repair recomputes whole rows: candidate room for the whole key axis
+    pl.rcap = candidate_capacity(topk, axis);
+    pl.off_rcand = off;
+    off += round_up(static_cast<int64_t>(2) * pl.rgrid * pl.R * pl.rcap * 8, 256);
+  } else {
+    pl.rcap = pl.cap;
+    pl.off_rcand = pl.off_cand;
   }
   pl.total = off;
 }
 
-// Row blocks of 8 rows; when they cannot fill the GPU, the key axis is cut
-// into chunks so that about two units land on every SM.
+// The fused top-k on a prepared plan: wires the workspace into `p` (whose
+// inputs, tensor maps and outputs are set), clears the per-call words, and
+// launches the indexer (and the merge when the key axis is split), then the
+// repair launch, which recomputes, exactly and whole, any row block or
+// request whose estimated threshold the checks rejected (it ends at once
+// when none was listed).
+int run_fused_topk(const Plan& pl, IndexerParams& p, uint8_t* wsb, bool paged, int R, int64_t rows,
+                   cudaStream_t st) {
+  const int topk = p.topk;
+  p.n_chunks = pl.n_chunks;
+  p.chunk_keys = pl.chunk_keys;
+  p.num_units = pl.num_units;
+  p.status = reinterpret_cast<int*>(wsb);
+  p.cand = reinterpret_cast<uint2*>(wsb + pl.off_cand);
+  p.cand_cap = pl.cap;
+  p.scratch = reinterpret_cast<uint2*>(wsb + pl.off_scratch);
+  p.repair_flag = reinterpret_cast<int*>(wsb + pl.off_repair);
+  p.repair_list = p.repair_flag + pl.groups;
+  p.speculate = 1;
+  p.repair_mode = 0;
+  p.wait_limit_ns = g_wait_limit_ns;
+  p.debug_withhold_first_tile = g_debug_withhold;
+  cudaError_t e = cudaMemsetAsync(p.repair_flag, 0, static_cast<size_t>(pl.groups) * 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "repair flags reset");
+  if (pl.n_chunks > 1) {
+    p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
+    p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
+    p.row_theta = reinterpret_cast<uint32_t*>(wsb + pl.off_theta);
+    p.row_spec = reinterpret_cast<uint32_t*>(wsb + pl.off_spec);
+    e = cudaMemsetAsync(p.row_theta, 0, pl.off_spec + round_up(static_cast<int64_t>(pl.groups) * pl.R * 4, 256) -
+                                            pl.off_theta, st);
+    if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
+  }
+  e = paged ? launch_indexer_paged_topk(p, R, pl.grid, st) : launch_indexer_prefill_topk(p, pl.grid, st);
+  if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
+  if (pl.n_chunks > 1) {
+    MergeParams mp{p.part, p.part_cnt, static_cast<int>(rows), pl.R, pl.n_chunks, topk, p.out_idx, p.out_vals,
+                   p.row_spec, p.status, p.repair_flag, p.repair_list};
+    e = launch_merge(mp, st);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  }
+  IndexerParams r = p;  // the repair: listed groups, whole rows, exact thresholds, direct output
+  r.repair_mode = 1;
+  r.speculate = 0;
+  r.n_chunks = 1;
+  r.chunk_keys = static_cast<int>(round_up(std::max<int64_t>(pl.axis, 1), kBlockKeys));
+  r.num_units = pl.groups;
+  r.cand = reinterpret_cast<uint2*>(wsb + pl.off_rcand);
+  r.cand_cap = pl.rcap;
+  r.part = nullptr;
+  r.part_cnt = nullptr;
+  r.row_theta = nullptr;
+  r.row_spec = nullptr;
+  r.debug_withhold_first_tile = 0;
+  e = paged ? launch_indexer_paged_topk(r, R, pl.rgrid, st) : launch_indexer_prefill_topk(r, pl.rgrid, st);
+  if (e != cudaSuccess) return cuda_fail(e, "repair launch");
+  return ok();
+}
+
+// Row blocks of kPrefillRows rows; when they cannot fill the GPU, the key
+// axis is cut into chunks so that about two units land on every SM.
 Plan plan_prefill(int64_t m, int64_t n, int topk, int sms) {
   Plan pl;
-  pl.R = 8;
+  pl.R = kPrefillRows;
   const int64_t groups = ceil_div(m, pl.R);
   const int64_t axis = std::max<int64_t>(n, 1);
   pl.chunk_keys = static_cast<int>(round_up(axis, kBlockKeys));
@@ -393,32 +471,9 @@ int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, c
   p.n = n;
   p.m = static_cast<int>(m);
   p.topk = topk;
-  p.n_chunks = pl.n_chunks;
-  p.chunk_keys = pl.chunk_keys;
-  p.num_units = pl.num_units;
   p.out_idx = out_idx;
   p.out_vals = out_vals;
-  p.status = reinterpret_cast<int*>(wsb);
-  p.cand = reinterpret_cast<uint2*>(wsb + pl.off_cand);
-  p.cand_cap = pl.cap;
-  p.scratch = reinterpret_cast<uint2*>(wsb + pl.off_scratch);
-  if (pl.n_chunks > 1) {
-    p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
-    p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
-    p.row_theta = reinterpret_cast<uint32_t*>(wsb + pl.off_theta);
-    e = cudaMemsetAsync(p.row_theta, 0, static_cast<size_t>(pl.num_units / pl.n_chunks) * pl.R * 4, st);
-    if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
-  }
-  p.wait_limit_ns = g_wait_limit_ns;
-  p.debug_withhold_first_tile = g_debug_withhold;
-  e = launch_indexer_prefill_topk(p, pl.grid, st);
-  if (e != cudaSuccess) return cuda_fail(e, "mqa_logits_topk launch");
-  if (pl.n_chunks > 1) {
-    MergeParams mp{p.part, p.part_cnt, static_cast<int>(m), pl.R, pl.n_chunks, topk, out_idx, out_vals};
-    e = launch_merge(mp, st);
-    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
-  }
-  return ok();
+  return run_fused_topk(pl, p, wsb, false, pl.R, m, st);
 }
 
 size_t fp8idx_paged_mqa_logits_topk_workspace(int64_t B, int R, int max_blocks, int H, int D,
@@ -482,32 +537,9 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
   p.max_blocks = max_blocks;
   p.num_pages = static_cast<int>(num_pages);
   p.topk = topk;
-  p.n_chunks = pl.n_chunks;
-  p.chunk_keys = pl.chunk_keys;
-  p.num_units = pl.num_units;
   p.out_idx = out_idx;
   p.out_vals = out_vals;
-  p.status = reinterpret_cast<int*>(wsb);
-  p.cand = reinterpret_cast<uint2*>(wsb + pl.off_cand);
-  p.cand_cap = pl.cap;
-  p.scratch = reinterpret_cast<uint2*>(wsb + pl.off_scratch);
-  if (pl.n_chunks > 1) {
-    p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
-    p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
-    p.row_theta = reinterpret_cast<uint32_t*>(wsb + pl.off_theta);
-    e = cudaMemsetAsync(p.row_theta, 0, static_cast<size_t>(pl.num_units / pl.n_chunks) * pl.R * 4, st);
-    if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
-  }
-  p.wait_limit_ns = g_wait_limit_ns;
-  p.debug_withhold_first_tile = g_debug_withhold;
-  e = launch_indexer_paged_topk(p, R, pl.grid, st);
-  if (e != cudaSuccess) return cuda_fail(e, "paged_mqa_logits_topk launch");
-  if (pl.n_chunks > 1) {
-    MergeParams mp{p.part, p.part_cnt, static_cast<int>(B * R), pl.R, pl.n_chunks, topk, out_idx, out_vals};
-    e = launch_merge(mp, st);
-    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
-  }
-  return ok();
+  return run_fused_topk(pl, p, wsb, true, R, B * R, st);
 }
 
 // Allocation-free form of fp8idx_mqa_logits_topk for callers that cannot
@@ -567,31 +599,10 @@ int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const flo
   p.n = n;
   p.m = static_cast<int>(m);
   p.topk = topk;
-  p.n_chunks = pl.n_chunks;
-  p.chunk_keys = pl.chunk_keys;
-  p.num_units = pl.num_units;
   p.out_idx = out_idx;
   p.out_vals = out_vals;
-  p.status = reinterpret_cast<int*>(wsb);
-  p.cand = reinterpret_cast<uint2*>(wsb + pl.off_cand);
-  p.cand_cap = pl.cap;
-  p.scratch = reinterpret_cast<uint2*>(wsb + pl.off_scratch);
-  if (pl.n_chunks > 1) {
-    p.part = reinterpret_cast<uint2*>(wsb + pl.off_part);
-    p.part_cnt = reinterpret_cast<int*>(wsb + pl.off_cnt);
-    p.row_theta = reinterpret_cast<uint32_t*>(wsb + pl.off_theta);
-    e = cudaMemsetAsync(p.row_theta, 0, static_cast<size_t>(pl.num_units / pl.n_chunks) * pl.R * 4, st);
-    if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
-  }
-  p.wait_limit_ns = g_wait_limit_ns;
-  p.debug_withhold_first_tile = g_debug_withhold;
-  e = launch_indexer_prefill_topk(p, pl.grid, st);
-  if (e != cudaSuccess) return cuda_fail(e, "mqa_logits_topk_noalloc launch");
-  if (pl.n_chunks > 1) {
-    MergeParams mp{p.part, p.part_cnt, static_cast<int>(m), pl.R, pl.n_chunks, topk, out_idx, out_vals};
-    e = launch_merge(mp, st);
-    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
-  }
+  const int rc = run_fused_topk(pl, p, wsb, false, pl.R, m, st);
+  if (rc != FP8IDX_OK) return rc;
   return ok();
 }
 

@@ -43,24 +43,33 @@
 
 namespace fp8idx {
 
+// Warp roles: warpgroup 0 holds the TMA producer (warp 0), the MMA issuer
+// (warp 1) and the select group (warps 2-3); then EWG epilogue warpgroups of
+// four warps, one per TMEM lane quadrant (warp % 4), each warpgroup owning RW
+// rows of the unit.  More epilogue warpgroups with fewer rows each give every
+// SM sub-partition more independent warps to hide the epilogue's latencies.
 template <int R, bool PAGED>
 struct Cfg {
   static constexpr int N = R * kHeads;         // MMA N: (row, head) columns
-  static constexpr int RW = R / 2;             // rows per epilogue warpgroup
+  static constexpr int RW = R == 8 ? 4 : 2;    // rows per epilogue warpgroup
+  static constexpr int EWG = R / RW;           // epilogue warpgroups
+  static constexpr int EPI_WARPS = 4 * EWG;
+  static constexpr int THREADS = 32 * (4 + EPI_WARPS);
   static constexpr int STAGES = PAGED ? (R == 8 ? 5 : 7) : 5;  // key-tile ring depth
   static constexpr int Q_BYTES = N * kDim;
   static constexpr int TILE_BYTES = kBlockKeys * kDim;
-  static constexpr int TMEM_COLS = 2 * N;
+  static constexpr int TMEM_COLS = 2 * N <= 256 ? 256 : 512;  // double-buffered accumulators
   static constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockKeys, N);
   static_assert(N <= 256 && N % 16 == 0, "MMA N out of range");
-  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns must be a power of two");
+  static_assert(R % RW == 0 && EPI_WARPS <= kMaxEpiWarps, "epilogue layout");
 };
 
 constexpr int kNB = 512;         // histogram bins per row
 constexpr int kSelWords = 264;   // per epilogue warp: hist[256], counter, pad
-constexpr int kSelWG = 10;       // first warp of the select group
+constexpr int kSelWG = 2;        // first warp of the select group
 constexpr int kSelWarps = 2;     // warps in the select group
-constexpr int kSelBar = 3;       // its named barrier
+constexpr int kEpiWG = 4;        // first epilogue warp
+constexpr int kSelBar = 8;       // the select group's named barrier (epilogue warpgroups use 1..EWG)
 constexpr int kUpCap = kMaxTopK; // per select warp: keys above the boundary bin (fewer than topk in all)
 constexpr int kAtCap = 1024;     // per select warp: keys inside the boundary bin
 constexpr int kSelBatch = 16;    // candidate loads in flight per select thread
@@ -72,9 +81,11 @@ constexpr int kSelBatch = 16;    // candidate loads in flight per select thread
 // barrier: the histogram is counted with shared-memory atomics, the window is
 // opened once by compare-and-swap, and the threshold only grows (atomicMax).
 struct RowState {
-  int wcnt[4];       // candidates in each segment (written when the unit ends)
-  uint32_t theta;    // lower bound on the row's k-th order key: keep a key iff key >= theta
-  int lo, hi;        // the row's key range inside this unit's chunk
+  int wcnt[4];          // candidates in each segment (written when the unit ends)
+  uint32_t theta;       // keep a key iff key >= theta (raised by bounds and by estimates)
+  uint32_t theta_spec;  // largest threshold raised by an estimate (0: none): checked after the select
+  int lo, hi;           // the row's key range inside this unit's chunk
+  int vtot;             // the row's valid keys over the whole key axis
   int pad;
   unsigned long long win;  // histogram window: base | shift << 32 | 1 << 40 once open
 };
@@ -121,7 +132,7 @@ __host__ __device__ constexpr SmemLayout smem_layout() {
   L.meta = L.rows + 2 * R * static_cast<int>(sizeof(RowState));
   L.hist = L.meta + 2 * static_cast<int>(sizeof(SlotMeta));
   L.esel = L.hist + 2 * R * kNB * 4;
-  L.ssel = L.esel + 8 * kSelWords * 4;
+  L.ssel = L.esel + C::EPI_WARPS * kSelWords * 4;
   L.up = L.ssel + 320 * 4;
   L.at = L.up + kSelWarps * kUpCap * 8;
   L.total = L.at + kSelWarps * kAtCap * 8;
@@ -281,6 +292,43 @@ __device__ __forceinline__ float relu_dot32_x2(const uint32_t (&x)[32], const fl
   unpack_f32x2(lin0, l0, l1);
   unpack_f32x2(lin1, l2, l3);
   return ((l0 + ab0) + (l1 + ab1)) + ((l2 + ab2) + (l3 + ab3));
+}
+
+// relu_dot32_x2 for two rows at once, written so that the two rows' twelve
+// accumulator chains interleave (an FMA waits on its own chain only).
+__device__ __forceinline__ void relu_dot32_x2_pair(const uint32_t (&xa)[32], const uint32_t (&xb)[32],
+                                                   const float* wa, const float* wb, float& ra, float& rb) {
+  const float4* wa4 = reinterpret_cast<const float4*>(wa);
+  const float4* wb4 = reinterpret_cast<const float4*>(wb);
+  uint64_t la0 = 0, la1 = 0, lb0 = 0, lb1 = 0;
+  float aa0 = 0.f, aa1 = 0.f, aa2 = 0.f, aa3 = 0.f, ab0 = 0.f, ab1 = 0.f, ab2 = 0.f, ab3 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 va = wa4[i], vb = wb4[i];
+    const float a0 = __uint_as_float(xa[4 * i + 0]), a1 = __uint_as_float(xa[4 * i + 1]);
+    const float a2 = __uint_as_float(xa[4 * i + 2]), a3 = __uint_as_float(xa[4 * i + 3]);
+    const float b0 = __uint_as_float(xb[4 * i + 0]), b1 = __uint_as_float(xb[4 * i + 1]);
+    const float b2 = __uint_as_float(xb[4 * i + 2]), b3 = __uint_as_float(xb[4 * i + 3]);
+    la0 = fma_f32x2(pack_f32x2(va.x, va.y), pack_f32x2(a0, a1), la0);
+    lb0 = fma_f32x2(pack_f32x2(vb.x, vb.y), pack_f32x2(b0, b1), lb0);
+    la1 = fma_f32x2(pack_f32x2(va.z, va.w), pack_f32x2(a2, a3), la1);
+    lb1 = fma_f32x2(pack_f32x2(vb.z, vb.w), pack_f32x2(b2, b3), lb1);
+    aa0 = fmaf(va.x, fabsf(a0), aa0);
+    ab0 = fmaf(vb.x, fabsf(b0), ab0);
+    aa1 = fmaf(va.y, fabsf(a1), aa1);
+    ab1 = fmaf(vb.y, fabsf(b1), ab1);
+    aa2 = fmaf(va.z, fabsf(a2), aa2);
+    ab2 = fmaf(vb.z, fabsf(b2), ab2);
+    aa3 = fmaf(va.w, fabsf(a3), aa3);
+    ab3 = fmaf(vb.w, fabsf(b3), ab3);
+  }
+  float a_l0, a_l1, a_l2, a_l3, b_l0, b_l1, b_l2, b_l3;
+  unpack_f32x2(la0, a_l0, a_l1);
+  unpack_f32x2(la1, a_l2, a_l3);
+  unpack_f32x2(lb0, b_l0, b_l1);
+  unpack_f32x2(lb1, b_l2, b_l3);
+  ra = ((a_l0 + aa0) + (a_l1 + aa1)) + ((a_l2 + aa2) + (a_l3 + aa3));
+  rb = ((b_l0 + ab0) + (b_l1 + ab1)) + ((b_l2 + ab2) + (b_l3 + ab3));
 }
 
 // (Only meaningful for key >= base; any other key maps to some bin in range.)
@@ -490,6 +538,33 @@ __device__ int final_select_row(const uint2* rowbuf, int wcap, const RowState& s
   });
 }
 
+// Minimum of one value per thread over a select group (xchg: two words of
+// scratch when the group has two warps).
+template <int G>
+__device__ __forceinline__ uint32_t group_min(uint32_t v, const Group<G>& g, uint32_t* xchg) {
+  v = __reduce_min_sync(0xFFFFFFFFu, v);
+  if (G > 1) {
+    g.sync();
+    if (g.lane() == 0) xchg[10 + g.warp()] = v;
+    g.sync();
+    v = min(xchg[10], xchg[11]);
+    g.sync();
+  }
+  return v;
+}
+
+// A row whose threshold was raised by an estimate: the result is the row's
+// top-k iff it is complete and its smallest key is at or above the largest
+// estimate applied (every key at or above that estimate passed every filter).
+// Otherwise the row's group (row block or request) is listed, once, for an
+// exact recomputation.
+__device__ __forceinline__ void check_estimate(const IndexerParams& p, int group, uint32_t spec, bool complete,
+                                               uint32_t kth_key, bool leader) {
+  if ((complete && kth_key >= spec) || !leader) return;
+  atomicAdd(p.status + kStatRepairs, 1);
+  if (atomicExch(p.repair_flag + group, 1) == 0) p.repair_list[atomicAdd(p.status + kRepairCount, 1)] = group;
+}
+
 // Exact top-k of one finished row (row rl of a slot) written out: the final
 // list (-1 / -inf padded) with one key chunk, else the unit's partial list and
 // its length.
@@ -507,15 +582,19 @@ __device__ void write_row_topk(const IndexerParams& p, const SlotMeta& meta, int
     const int row = meta.row0 + rl;
     int32_t* orow = p.out_idx + static_cast<int64_t>(row) * k;
     float* vrow = p.out_vals ? p.out_vals + static_cast<int64_t>(row) * k : nullptr;
+    uint32_t vmin = 0xFFFFFFFFu;  // the smallest order key written (this thread's share)
     const int nout = final_select_row<FAST>(rowbuf, wcap, st, h, k, g, up_all, at_all, xchg, p.status,
                                             [&](int pos, uint32_t key, uint32_t j) {
                                               orow[pos] = static_cast<int32_t>(j);
                                               if (vrow) vrow[pos] = key_to_float(key);
+                                              vmin = min(vmin, key);
                                             });
     for (int pos = nout + g.tid; pos < k; pos += 32 * G) {
       orow[pos] = -1;
       if (vrow) vrow[pos] = -INFINITY;
     }
+    if (st.theta_spec != 0u)
+      check_estimate(p, meta.unit, st.theta_spec, nout >= min(k, st.vtot), group_min(vmin, g, xchg), g.tid == 0);
   } else {
     uint2* prow = p.part + (static_cast<size_t>(meta.unit) * R + rl) * k;
     int nout = 0;
@@ -543,6 +622,7 @@ __device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned lon
 __device__ __forceinline__ uint32_t ld_volatile_u32(const uint32_t* p) {
   return *reinterpret_cast<const volatile uint32_t*>(p);
 }
+__device__ __forceinline__ int ld_volatile_i32(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
 
 // Count candidates [from, to) of one warp's segment of a row into the row's
 // histogram.  If the row's window is not open yet (then from == 0: nothing of
@@ -642,31 +722,51 @@ __device__ __forceinline__ int compact_segment(uint2* seg, int cnt, int room, in
   return kept;
 }
 
-// Raise a row's threshold to the lower edge of the histogram bin that holds
-// the k-th counted key (at least k keys of the row lie at or above it).  With
-// the key axis split over several units, the bound is shared through the
-// row's word in global memory: any unit's bound is a bound for the whole row.
-__device__ __forceinline__ void raise_theta(const uint32_t* h, RowState* st, int k, uint32_t* row_theta,
-                                         int lane) {
+// Raise a row's threshold from its histogram.  Exact: to the lower edge of
+// the bin that holds the k-th counted key (at least k keys of the row lie at
+// or above it).  Estimated (target < k): to the lower edge of the bin that
+// holds the target-th counted key, where the target is the expected number
+// of the row's top-k among the keys seen so far plus a five-sigma margin; the
+// result is then recorded as an estimate to be checked after the select.
+// With the key axis split over several units, thresholds are shared through
+// the row's words in global memory (any unit's bound is a bound for the
+// whole row; estimates are recorded there too).
+__device__ __forceinline__ void raise_theta(const uint32_t* h, RowState* st, int target, bool estimate,
+                                            uint32_t* row_theta, uint32_t* row_spec, int lane) {
   const Window w = window_of(ld_volatile_u64(&st->win));
   uint32_t th = 0;
   if (w.open) {
-    const Boundary B = find_boundary(h, static_cast<uint32_t>(k), lane);
+    const Boundary B = find_boundary(h, static_cast<uint32_t>(target), lane);
     if (B.found) {
       const uint64_t t64 = static_cast<uint64_t>(w.base) + (static_cast<uint64_t>(B.bin) << w.shift);
       th = t64 > 0xFFFFFFFFull ? 0xFFFFFFFFu : static_cast<uint32_t>(t64);
     }
   }
   if (lane == 0) {
+    if (estimate && th) {
+      atomicMax(&st->theta_spec, th);
+      if (row_spec) atomicMax(row_spec, th);
+    }
     if (row_theta) th = max(th, atomicMax(row_theta, th));
     if (th) atomicMax(&st->theta, th);
   }
 }
 
+// The target count of an estimated threshold after `seen` of a row's `vtot`
+// keys: mean + 5 sqrt(mean) + 8 with mean = k * seen / vtot (the expected
+// number of the row's top-k among keys seen in random order).  Returns k
+// (exact) when the estimate would not be below the exact bound.
+__device__ __forceinline__ int estimate_target(int k, int seen, int vtot) {
+  if (vtot <= k || seen <= 0) return k;
+  const float mean = static_cast<float>(k) * static_cast<float>(seen) / static_cast<float>(vtot);
+  const float c = ceilf(mean + 5.0f * sqrtf(mean) + 8.0f);
+  return c < static_cast<float>(min(k, seen)) ? static_cast<int>(c) : k;
+}
+
 // ------------------------------------------------------------------ kernel
 
 template <int R, bool PAGED, int MODE>
-__global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_constant__ IndexerParams p) {
+__global__ void __launch_bounds__(Cfg<R, PAGED>::THREADS, 1) indexer_kernel(const __grid_constant__ IndexerParams p) {
   using C = Cfg<R, PAGED>;
   constexpr SmemLayout SL = smem_layout<R, PAGED>();
   constexpr int N = C::N;
@@ -708,6 +808,9 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // a repair launch with nothing listed ends at once (the count is final: the
+  // launches that list groups ran before this one on the stream)
+  if (p.repair_mode && ld_volatile_i32(p.status + kRepairCount) == 0) return;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -716,13 +819,13 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);
-      mbar_init(&slot_full[a], 8);
+      mbar_init(&tempty[a], C::EPI_WARPS);
+      mbar_init(&slot_full[a], C::EPI_WARPS);
       mbar_init(&slot_empty[a], kSelWarps);
     }
     for (int x = 0; x < 4; ++x) {
       mbar_init(&uq_full[x], 1);
-      mbar_init(&uq_empty[x], 9);  // the MMA thread and the eight epilogue warps
+      mbar_init(&uq_empty[x], 1 + C::EPI_WARPS);  // the MMA thread and every epilogue warp
     }
     mbar_init(qfull, 1);
     mbar_init(qempty, 1);
@@ -766,12 +869,17 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       for (int n = 0; ok; ++n) {
         const int qs = n & 3;
         if (!wait_phase<kSleep>(&uq_empty[qs], ((n >> 2) & 1) ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
-        const int idx = atomicAdd(p.status + kSchedWord, 1);
         int u = -1;
-        if (idx < p.num_units) {
-          const int groups = p.num_units / p.n_chunks;
-          u = p.n_chunks == 1 ? p.num_units - 1 - idx
-                              : (groups - 1 - idx % groups) * p.n_chunks + idx / groups;
+        if (p.repair_mode) {  // the groups the checks listed, one unit each (whole rows)
+          const int idx = atomicAdd(p.status + kRepairSched, 1);
+          if (idx < ld_volatile_i32(p.status + kRepairCount)) u = p.repair_list[idx];
+        } else {
+          const int idx = atomicAdd(p.status + kSchedWord, 1);
+          if (idx < p.num_units) {
+            const int groups = p.num_units / p.n_chunks;
+            u = p.n_chunks == 1 ? p.num_units - 1 - idx
+                                : (groups - 1 - idx % groups) * p.n_chunks + idx / groups;
+          }
         }
         uq[qs] = u;
         mbar_arrive(&uq_full[qs]);
@@ -871,9 +979,9 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         }
       }
     }
-  } else if (warp < kSelWG) {
+  } else if (warp >= kEpiWG) {
     // ---------------------------------------------------------------- epilogue
-    const int ew = warp - 2;  // 0..7
+    const int ew = warp - kEpiWG;  // 0 .. EPI_WARPS - 1
     const int g = ew >> 2;    // warpgroup
     const int qd = warp & 3;  // TMEM lane quadrant == key block of 32 == buffer segment
     const int tid_wg = qd * 32 + lane;
@@ -948,7 +1056,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
       // (kept in shared memory; the tile loop reads it back as a broadcast)
       if (tid_wg < RW) {
         const int rl = g * RW + tid_wg;
-        int lo = 0, hi = 0;
+        int lo = 0, hi = 0, vtot = 0;
         if (rl < U.nrows) {
           const int row = U.row0 + rl;
           if (!PAGED) {
@@ -958,12 +1066,14 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
             const int e = U.len - R + rl + 1;
             hi = max(min(e, U.len), 0);
           }
+          vtot = hi - lo;
           // a unit only owns the keys of its chunk (its last tile may overhang)
           lo = max(lo, U.cbeg);
           hi = max(lo, min(hi, U.cend));
         }
         rs[tid_wg].lo = lo;
         rs[tid_wg].hi = hi;
+        rs[tid_wg].vtot = vtot;
       }
       if (tid_wg < RW * kHeads) {
         const int rl = g * RW + tid_wg / kHeads;
@@ -974,6 +1084,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
           RowState& st = rs[tid_wg];
           st.wcnt[0] = st.wcnt[1] = st.wcnt[2] = st.wcnt[3] = 0;
           st.theta = 0;
+          st.theta_spec = 0;
           st.win = 0ull;
         }
         for (int x = tid_wg; x < RW * kNB; x += 128) hs[x] = 0;
@@ -1041,22 +1152,37 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
         const uint32_t a = T & 1, aph = (T >> 1) & 1;
         if (!wait_phase<kSpin>(&tfull[a], aph, abort_flag, p.status, limit)) aborted = true;
         tc_fence_after();
+        // Rows in pairs (64 TMEM columns per pair); the next pair's loads are
+        // in flight while the current pair's sums are formed.  The last wait
+        // leaves the whole accumulator in registers: release it to the MMA.
+        // (fma with +0: an exactly zero head sum gives +0 whatever the sign
+        // of the scale.)
+        static_assert(RW == 2 || RW == 4, "rows per warpgroup");
         float L[RW];
-#pragma unroll
-        for (int r = 0; r < RW; r += 2) {  // two rows (64 columns) per TMEM read
-          uint32_t x0[32], x1[32];
-          tmem_ld32(lane_addr + a * N + (g * RW + r) * kHeads, x0);
-          tmem_ld32(lane_addr + a * N + (g * RW + r + 1) * kHeads, x1);
+        {
+          uint32_t xa[32], xb[32];
+          tmem_ld32(lane_addr + a * N + (g * RW + 0) * kHeads, xa);
+          tmem_ld32(lane_addr + a * N + (g * RW + 1) * kHeads, xb);
           tmem_ld_wait();
-          if (r + 2 == RW) {  // the accumulator is in registers now
+          if (RW == 2) {
             tc_fence_before();
             __syncwarp();
             mbar_arrive_if(lane == 0, &tempty[a]);
+            relu_dot32_x2_pair(xa, xb, ws_g, ws_g + kHeads, L[0], L[1]);
+          } else {
+            uint32_t xc[32], xd[32];
+            tmem_ld32(lane_addr + a * N + (g * RW + 2) * kHeads, xc);
+            tmem_ld32(lane_addr + a * N + (g * RW + 3) * kHeads, xd);
+            relu_dot32_x2_pair(xa, xb, ws_g, ws_g + kHeads, L[0], L[1]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            mbar_arrive_if(lane == 0, &tempty[a]);
+            relu_dot32_x2_pair(xc, xd, ws_g + 2 * kHeads, ws_g + 3 * kHeads, L[2], L[RW - 1]);
           }
-          // fma with +0: an exactly zero head sum gives +0 whatever the sign of the scale
-          L[r] = fmaf(relu_dot32_x2(x0, ws_g + r * kHeads), sj, 0.f);
-          L[r + 1] = fmaf(relu_dot32_x2(x1, ws_g + (r + 1) * kHeads), sj, 0.f);
         }
+#pragma unroll
+        for (int r = 0; r < RW; ++r) L[r] = fmaf(L[r], sj, 0.f);
 
         if (MODE == kModeLogits) {
 #pragma unroll
@@ -1068,18 +1194,32 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
           if (aborted) break;
         } else {
           // ---- filter against the row's threshold; append to this warp's segment
-          // and count the key into the row's histogram (once its window is open)
+          // and count the key into the row's histogram (once its window is open).
+          // Stage by stage over the rows, so that the rows' chains interleave
+          // ahead of the stores (which keep their order).
+          bool ps[RW];
+          uint32_t key[RW], msk[RW];
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
-            const bool ps = static_cast<uint32_t>(j - lo[r]) < static_cast<uint32_t>(span[r]) && L[r] >= thf[r];
-            const uint32_t msk = __ballot_sync(0xFFFFFFFFu, ps);
-            const int pos = cnt[r] + __popc(msk & lt);
-            cnt[r] += __popc(msk);
-            const uint32_t key = order_key_nz(L[r]);
-            st_global_v2_if(ps && pos < wcap, seg0 + static_cast<size_t>(r) * cap + pos, key,
-                            static_cast<uint32_t>(j));
-            red_shared_add_if(ps && key >= hbase[r], hs + r * kNB + hist_bin(key, hbase[r], hshift[r]), 1u);
+            ps[r] = static_cast<uint32_t>(j - lo[r]) < static_cast<uint32_t>(span[r]) && L[r] >= thf[r];
+            key[r] = order_key_nz(L[r]);
           }
+#pragma unroll
+          for (int r = 0; r < RW; ++r) msk[r] = __ballot_sync(0xFFFFFFFFu, ps[r]);
+          int pos[RW];
+          uint32_t* hp[RW];
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            pos[r] = cnt[r] + __popc(msk[r] & lt);
+            cnt[r] += __popc(msk[r]);
+            hp[r] = hs + r * kNB + hist_bin(key[r], hbase[r], hshift[r]);
+          }
+#pragma unroll
+          for (int r = 0; r < RW; ++r)
+            st_global_v2_if(ps[r] && pos[r] < wcap, seg0 + static_cast<size_t>(r) * cap + pos[r], key[r],
+                            static_cast<uint32_t>(j));
+#pragma unroll
+          for (int r = 0; r < RW; ++r) red_shared_add_if(ps[r] && key[r] >= hbase[r], hp[r], 1u);
           // ---- vote: count, make room, reload the thresholds (this warp alone)
           if (t == next_vote || t + 1 == U.ntiles) {
             const int vnext = vote_interval(t + 1);
@@ -1115,16 +1255,28 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_kernel(const __grid_const
                   cc = cnt[r];
                 }
               if (cr < 0) break;
-              uint2* scr = p.scratch + (static_cast<size_t>(blockIdx.x) * 8 + ew) * k;
+              uint2* scr = p.scratch + (static_cast<size_t>(blockIdx.x) * kMaxEpiWarps + ew) * k;
               const int nc = compact_segment(seg0 + static_cast<size_t>(cr) * cap, cc, room, wcap, k, rs + cr, scr,
                                              grp, p.status, lane);
 #pragma unroll
               for (int r = 0; r < RW; ++r)
                 if (r == cr) cnt[r] = folded[r] = nc;
             }
-            if (qd < RW && g * RW + qd < U.nrows)
-              raise_theta(hs + qd * kNB, rs + qd, k, p.n_chunks > 1 ? p.row_theta + U.row0 + g * RW + qd : nullptr,
-                          lane);
+            if (qd < RW && g * RW + qd < U.nrows) {
+              // this warp keeps the threshold of the group's row qd; an estimate
+              // counts the row's keys in tiles [0, t + 1] as seen (the other
+              // warps may be a tile ahead), which only lowers it
+              const RowState* me = rs + qd;
+              int target = k;
+              if (p.speculate) {
+                const int mlo = ld_volatile_i32(&me->lo), mhi = ld_volatile_i32(&me->hi);
+                const int seen = min(mhi, U.jbeg + (t + 2) * kBlockKeys) - max(mlo, U.jbeg);
+                target = estimate_target(k, max(0, min(seen, mhi - mlo)), ld_volatile_i32(&me->vtot));
+              }
+              const int row = U.row0 + g * RW + qd;
+              raise_theta(hs + qd * kNB, rs + qd, target, target < k, p.n_chunks > 1 ? p.row_theta + row : nullptr,
+                          p.n_chunks > 1 ? p.row_spec + row : nullptr, lane);
+            }
 #pragma unroll
             for (int r = 0; r < RW; ++r) thf[r] = theta_float(ld_volatile_u32(&rs[r].theta));
           }
@@ -1269,9 +1421,11 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
   }
   int32_t* orow = p.out_idx + static_cast<int64_t>(row) * p.topk;
   float* vrow = p.out_vals ? p.out_vals + static_cast<int64_t>(row) * p.topk : nullptr;
+  uint32_t vmin = 0xFFFFFFFFu;  // the smallest order key written (this thread's share)
   auto emit = [&](int pos, uint64_t K) {
     orow[pos] = static_cast<int32_t>(composite_index(K));
     if (vrow) vrow[pos] = key_to_float(composite_value(K));
+    vmin = min(vmin, composite_value(K));
   };
   int nout;
   if (total >= 0 && total <= kMergeStage) {
@@ -1293,6 +1447,24 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
   for (int pos = nout + threadIdx.x; pos < p.topk; pos += blockDim.x) {
     orow[pos] = -1;
     if (vrow) vrow[pos] = -INFINITY;
+  }
+  // A row whose threshold was raised by an estimate (only rows with more than
+  // topk keys): complete, with its smallest key at or above the largest
+  // estimate applied, or its request is listed for an exact recomputation.
+  const uint32_t spec = p.row_spec ? p.row_spec[row] : 0u;
+  if (spec != 0u) {
+    vmin = __reduce_min_sync(0xFFFFFFFFu, vmin);
+    if (lane == 0) red[warp] = vmin;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t m = 0xFFFFFFFFu;
+      for (int w = 0; w < kMergeWarps; ++w) m = min(m, red[w]);
+      if (nout < p.topk || m < spec) {
+        atomicAdd(p.status + kStatRepairs, 1);
+        if (atomicExch(p.repair_flag + unit_row, 1) == 0)
+          p.repair_list[atomicAdd(p.status + kRepairCount, 1)] = unit_row;
+      }
+    }
   }
 }
 
@@ -1345,15 +1517,15 @@ static cudaError_t launch_indexer(const IndexerParams& p, int grid, cudaStream_t
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, st>>>(p);
+  kern<<<grid, Cfg<R, PAGED>::THREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_indexer_prefill_logits(const IndexerParams& p, int grid, cudaStream_t st) {
-  return launch_indexer<8, false, kModeLogits>(p, grid, st);
+  return launch_indexer<kPrefillRows, false, kModeLogits>(p, grid, st);
 }
 cudaError_t launch_indexer_prefill_topk(const IndexerParams& p, int grid, cudaStream_t st) {
-  return launch_indexer<8, false, kModeTopK>(p, grid, st);
+  return launch_indexer<kPrefillRows, false, kModeTopK>(p, grid, st);
 }
 cudaError_t launch_indexer_paged_topk(const IndexerParams& p, int R, int grid, cudaStream_t st) {
   if (R == 8) return launch_indexer<8, true, kModeTopK>(p, grid, st);

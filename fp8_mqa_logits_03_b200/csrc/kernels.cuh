@@ -12,7 +12,8 @@ constexpr int kDim = 128;          // index head dim (bytes per fp8 row)
 constexpr int kBlockKeys = 128;    // keys per tile = MMA M = TMEM lanes
 constexpr int kPageSize = 64;      // tokens per key page (paged form)
 constexpr int kMaxTopK = 2048;
-constexpr int kThreads = 384;      // 12 warps: TMA, MMA, 8 epilogue, 2 select
+constexpr int kPrefillRows = 6;    // query rows per prefill unit (row block)
+constexpr int kMaxEpiWarps = 12;   // epilogue warps per CTA at most (workspace scratch is sized for it)
 constexpr int kStatusBytes = 256;  // device status block at the head of every workspace
 // Tiles between two group votes of the fused epilogue, after t tiles of the
 // unit: short early, where the running threshold still moves fast, and
@@ -34,7 +35,11 @@ constexpr int kStatCompactions = 1;     // in-stream exact compactions of a full
 constexpr int kStatGeneralSelects = 2;  // final selects that needed the general radix path
 constexpr int kStatCandidates = 3;      // candidates appended, summed over rows
 constexpr int kStatMaxBoundary = 4;     // largest boundary-bin population seen
+constexpr int kStatRepairs = 5;         // rows whose estimated threshold proved too high (recomputed exactly)
 constexpr int kSchedWord = 16;          // status-block word: next unit for dynamic scheduling
+constexpr int kRepairCount = 18;        // status-block word: row blocks / requests listed for recomputation
+constexpr int kRepairSched = 19;        // status-block word: next listed group for the repair launch
+constexpr int kRepairMaxGrid = 32;      // CTAs of a repair launch at most
 
 enum Mode : int { kModeLogits = 0, kModeTopK = 1 };
 
@@ -65,12 +70,20 @@ struct IndexerParams {
   int* status;
   uint2* cand;      // [gridDim.x][2 slots][R][cand_cap] (order key, index); cand_cap % 128 == 0
   int cand_cap;     // per row; split into 4 equal segments, one per key quadrant
-  uint2* scratch;   // [gridDim.x][8 epilogue warps][topk]: staging of a rare in-kernel compaction
+  uint2* scratch;   // [gridDim.x][kMaxEpiWarps][topk]: staging of a rare in-kernel compaction
   uint2* part;      // split mode: [num_units][R][topk]
   int* part_cnt;    // split mode: [num_units][R]
   uint32_t* row_theta;  // split mode: [m] best lower bound on each row's k-th order key, zeroed per call
   unsigned long long wait_limit_ns;
   int debug_withhold_first_tile;  // tests only: never issue the first key tile's load (its wait runs out)
+  // estimated thresholds: a row's threshold may be raised to an estimate of
+  // its k-th value from the keys seen so far; the select (or the merge) checks
+  // the estimate against the result and lists the group for recomputation
+  int speculate;
+  uint32_t* row_spec;   // split mode: [m] largest estimated threshold applied to each row
+  int* repair_flag;     // [row blocks / requests]: listed for recomputation (zeroed per call)
+  int* repair_list;     // [row blocks / requests]
+  int repair_mode;      // this launch recomputes the listed groups, whole rows, exact thresholds
 };
 
 struct MergeParams {
@@ -82,6 +95,10 @@ struct MergeParams {
   int topk;
   int32_t* out_idx;
   float* out_vals;
+  const uint32_t* row_spec;  // [rows] largest estimated threshold applied (0: none; NULL: no estimates)
+  int* status;               // the call's status block (repair count and stats)
+  int* repair_flag;
+  int* repair_list;
 };
 
 struct TopkRowsParams {

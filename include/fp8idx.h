@@ -248,7 +248,9 @@ int fp8idx_read_device_status(const void* ws, int* status_out, void* stream);
  * word 1 the in-kernel compactions of a full candidate buffer, word 2 the rows
  * whose final selection took the general radix path, word 3 the candidates
  * collected (summed over rows and key chunks), word 4 the largest
- * boundary-bin population.  Synchronises `stream`; for tuning and tests. */
+ * boundary-bin population, word 5 the rows whose estimated threshold the
+ * check rejected (their row block or request was recomputed exactly).
+ * Synchronises `stream`; for tuning and tests. */
 int fp8idx_read_device_stats(const void* ws, uint32_t* out, int count, void* stream);
 /* Message for the last non-OK return on this thread ("" if none). */
 const char* fp8idx_last_error(void);

@@ -252,3 +252,47 @@ def test_paged_full_workload_sampled():
     assert fx.read_device_status(ws) == 0
     rows = _sample_rows(d["B"] * d["R"], 24, 4)
     _paged_check(d, idx.cpu().numpy(), vals.cpu().numpy(), rows, workloads.TOPK)
+
+
+# ---------------------------------------------------------------------------- estimated thresholds
+
+def _decaying_scales(n, rate):
+    """Key scales that fall along the key axis: the first keys seen dominate,
+    so a threshold estimated from them overshoots the row's k-th value."""
+    return (1.5 * torch.exp(-rate * torch.arange(n, dtype=torch.float64))).to(torch.float32) + 1e-3
+
+
+@pytest.mark.parametrize("m,n,k", [(40, 20000, 512), (6 * 148 + 3, 6000, 256)])  # split + merge; direct
+def test_fused_estimate_rejected_and_repaired(m, n, k):
+    """Adversarial key order: the estimate check rejects rows, their row blocks
+    are recomputed exactly, and every row still matches the oracle."""
+    d = workloads.make_prefill(m, n, 51)
+    d["s"] = _decaying_scales(n, 6.0 / n)
+    t = _to(d)
+    ws = fx.alloc_workspace(fx.mqa_logits_topk_workspace_size(m, n, k))
+    idx, vals = fx.mqa_logits_topk(**t, topk=k, return_values=True, workspace=ws)
+    stats = fx.read_device_stats(ws)
+    assert stats["status"] == 0
+    assert stats["repairs"] > 0, stats
+    rows = np.arange(m) if m <= 64 else np.concatenate([np.arange(0, 24), np.arange(m - 24, m)])
+    _check_fused(d, idx.cpu().numpy(), vals.cpu().numpy(), rows, k)
+
+
+def test_paged_estimate_rejected_and_repaired():
+    lengths = [9000, 4000, 12000, 700]
+    R, k = 4, 512
+    d = workloads.make_paged(len(lengths), R, 1, 12000, seed=52, lengths=lengths)
+    # scales falling with each request's logical position, written through its block table
+    sp = d["s_pages"].clone().view(-1)
+    for b, L in enumerate(lengths):
+        pos = torch.arange(L)
+        slots = d["block_table"][b, pos // 64].long() * 64 + pos % 64
+        sp[slots] = _decaying_scales(L, 6.0 / L)
+    d["s_pages"] = sp.view_as(d["s_pages"])
+    t = {key: d[key].cuda() for key in ("q", "k_pages", "s_pages", "w", "block_table", "seq_lens")}
+    ws = fx.alloc_workspace(fx.paged_workspace_size(len(lengths), R, d["max_blocks"], k))
+    idx, vals = fx.paged_mqa_logits_topk(**t, R=R, topk=k, return_values=True, workspace=ws)
+    stats = fx.read_device_stats(ws)
+    assert stats["status"] == 0
+    assert stats["repairs"] > 0, stats
+    _paged_check(d, idx.cpu().numpy(), vals.cpu().numpy(), np.arange(len(lengths) * R), k)
