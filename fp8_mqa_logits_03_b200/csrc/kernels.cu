@@ -730,9 +730,13 @@ __device__ __forceinline__ int compact_segment(uint2* seg, int cnt, int room, in
 // result is then recorded as an estimate to be checked after the select.
 // With the key axis split over several units, thresholds are shared through
 // the row's words in global memory (any unit's bound is a bound for the
-// whole row; estimates are recorded there too).
+// whole row; estimates are recorded there too): this unit's bound goes out as
+// a reduction that returns nothing, and the row's word is read without
+// waiting, its value taken up at the next vote (`gseen`), so that no vote
+// waits on a round trip to L2.
 __device__ __forceinline__ void raise_theta(const uint32_t* h, RowState* st, int target, bool estimate,
-                                            uint32_t* row_theta, uint32_t* row_spec, int lane) {
+                                            uint32_t* row_theta, uint32_t* row_spec, uint32_t& gseen,
+                                            int lane) {
   const Window w = window_of(ld_volatile_u64(&st->win));
   uint32_t th = 0;
   if (w.open) {
@@ -747,7 +751,11 @@ __device__ __forceinline__ void raise_theta(const uint32_t* h, RowState* st, int
       atomicMax(&st->theta_spec, th);
       if (row_spec) atomicMax(row_spec, th);
     }
-    if (row_theta) th = max(th, atomicMax(row_theta, th));
+    if (row_theta) {
+      if (th) atomicMax(row_theta, th);
+      th = max(th, gseen);
+      gseen = ld_volatile_u32(row_theta);
+    }
     if (th) atomicMax(&st->theta, th);
   }
 }
@@ -1133,6 +1141,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED>::THREADS, 1) indexer_kernel(cons
         hshift[r] = 0;
       }
       uint2* seg0 = MODE == kModeTopK ? cand_s + qd * wcap : nullptr;  // row r's segment: seg0 + r * cap
+      uint32_t gseen = 0;  // split key axis: the row's shared bound as read at this warp's last vote
 
       // ---- stream the unit's key tiles
       const int key0 = U.jbeg + qd * 32 + lane;
@@ -1275,7 +1284,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED>::THREADS, 1) indexer_kernel(cons
               }
               const int row = U.row0 + g * RW + qd;
               raise_theta(hs + qd * kNB, rs + qd, target, target < k, p.n_chunks > 1 ? p.row_theta + row : nullptr,
-                          p.n_chunks > 1 ? p.row_spec + row : nullptr, lane);
+                          p.n_chunks > 1 ? p.row_spec + row : nullptr, gseen, lane);
             }
 #pragma unroll
             for (int r = 0; r < RW; ++r) thf[r] = theta_float(ld_volatile_u32(&rs[r].theta));

@@ -12,7 +12,7 @@ constexpr int kDim = 128;          // index head dim (bytes per fp8 row)
 constexpr int kBlockKeys = 128;    // keys per tile = MMA M = TMEM lanes
 constexpr int kPageSize = 64;      // tokens per key page (paged form)
 constexpr int kMaxTopK = 2048;
-constexpr int kPrefillRows = 6;    // query rows per prefill unit (row block)
+constexpr int kPrefillRows = 8;    // query rows per prefill unit (row block)
 constexpr int kMaxEpiWarps = 12;   // epilogue warps per CTA at most (workspace scratch is sized for it)
 constexpr int kStatusBytes = 256;  // device status block at the head of every workspace
 // Tiles between two group votes of the fused epilogue, after t tiles of the
