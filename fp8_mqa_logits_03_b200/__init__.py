@@ -194,12 +194,12 @@ def topk_rows(logits, ks, ke, topk: int = MAX_TOPK, out=None, n=None, stream=Non
     return out
 
 
-def mqa_logits_topk_workspace_size(m: int, n: int, topk: int = MAX_TOPK) -> int:
-    return int(lib().fp8idx_mqa_logits_topk_workspace(m, n, H, D, topk))
+def mqa_logits_topk_workspace_size(m: int, n: int, topk: int = MAX_TOPK, heads: int = H) -> int:
+    return int(lib().fp8idx_mqa_logits_topk_workspace(m, n, heads, D, topk))
 
 
-def paged_workspace_size(B: int, R: int, max_blocks: int, topk: int = MAX_TOPK) -> int:
-    return int(lib().fp8idx_paged_mqa_logits_topk_workspace(B, R, max_blocks, H, D, topk))
+def paged_workspace_size(B: int, R: int, max_blocks: int, topk: int = MAX_TOPK, heads: int = H) -> int:
+    return int(lib().fp8idx_paged_mqa_logits_topk_workspace(B, R, max_blocks, heads, D, topk))
 
 
 def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
@@ -222,7 +222,7 @@ def mqa_logits_topk(q, k, s, w, ks, ke, topk: int = MAX_TOPK, out=None, out_vals
         out = torch.empty((m, topk), dtype=torch.int32, device=q.device)
     if return_values and out_vals is None:
         out_vals = torch.empty((m, topk), dtype=torch.float32, device=q.device)
-    need = mqa_logits_topk_workspace_size(m, n, topk)
+    need = mqa_logits_topk_workspace_size(m, n, topk, q.shape[1])
     if workspace is None:
         workspace = alloc_workspace(need, q.device)
     _check(lib().fp8idx_mqa_logits_topk(_ptr(q), _ptr(k), _ptr(s), _ptr(w), _ptr(ks), _ptr(ke), m,
@@ -251,7 +251,7 @@ def paged_mqa_logits_topk(q, k_pages, s_pages, w, block_table, seq_lens, R: int,
         out = torch.empty((rows, topk), dtype=torch.int32, device=q.device)
     if return_values and out_vals is None:
         out_vals = torch.empty((rows, topk), dtype=torch.float32, device=q.device)
-    need = paged_workspace_size(B, R, max_blocks, topk)
+    need = paged_workspace_size(B, R, max_blocks, topk, q.shape[1])
     if workspace is None:
         workspace = alloc_workspace(need, q.device)
     _check(lib().fp8idx_paged_mqa_logits_topk(_ptr(q), _ptr(k_pages), _ptr(s_pages), _ptr(w),

@@ -118,7 +118,9 @@ int make_rows128_map(CUtensorMap* map, const void* base, int64_t rows, int box_r
 // ---------------------------------------------------------------- plans
 
 struct Plan {
-  int R = 8;
+  int R = 8;           // the kernel's row capacity per unit (its MMA rows)
+  int rows_per_unit = 8;  // query rows of a row block / request (<= R)
+  int H = 32;
   int n_chunks = 1;
   int chunk_keys = 0;
   int num_units = 0;
@@ -190,8 +192,7 @@ void finish_plan(Plan& pl, int64_t groups, int sms, int topk, int64_t axis) {
 // repair launch, which recomputes, exactly and whole, any row block or
 // request whose estimated threshold the checks rejected (it ends at once
 // when none was listed).
-int run_fused_topk(const Plan& pl, IndexerParams& p, uint8_t* wsb, bool paged, int R, int64_t rows,
-                   cudaStream_t st) {
+int run_fused_topk(const Plan& pl, IndexerParams& p, uint8_t* wsb, bool paged, int64_t rows, cudaStream_t st) {
   const int topk = p.topk;
   p.n_chunks = pl.n_chunks;
   p.chunk_keys = pl.chunk_keys;
@@ -217,11 +218,12 @@ int run_fused_topk(const Plan& pl, IndexerParams& p, uint8_t* wsb, bool paged, i
                                             pl.off_theta, st);
     if (e != cudaSuccess) return cuda_fail(e, "threshold reset");
   }
-  e = paged ? launch_indexer_paged_topk(p, R, pl.grid, st) : launch_indexer_prefill_topk(p, pl.grid, st);
+  p.rows_per_unit = pl.rows_per_unit;
+  e = paged ? launch_indexer_paged_topk(p, pl.R, pl.H, pl.grid, st) : launch_indexer_prefill_topk(p, pl.H, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
   if (pl.n_chunks > 1) {
-    MergeParams mp{p.part, p.part_cnt, static_cast<int>(rows), pl.R, pl.n_chunks, topk, p.out_idx, p.out_vals,
-                   p.row_spec, p.status, p.repair_flag, p.repair_list};
+    MergeParams mp{p.part, p.part_cnt, static_cast<int>(rows), pl.rows_per_unit, pl.R, pl.n_chunks, topk,
+                   p.out_idx, p.out_vals, p.row_spec, p.status, p.repair_flag, p.repair_list};
     e = launch_merge(mp, st);
     if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }
@@ -238,16 +240,19 @@ int run_fused_topk(const Plan& pl, IndexerParams& p, uint8_t* wsb, bool paged, i
   r.row_theta = nullptr;
   r.row_spec = nullptr;
   r.debug_withhold_first_tile = 0;
-  e = paged ? launch_indexer_paged_topk(r, R, pl.rgrid, st) : launch_indexer_prefill_topk(r, pl.rgrid, st);
+  e = paged ? launch_indexer_paged_topk(r, pl.R, pl.H, pl.rgrid, st) : launch_indexer_prefill_topk(r, pl.H, pl.rgrid, st);
   if (e != cudaSuccess) return cuda_fail(e, "repair launch");
   return ok();
 }
 
-// Row blocks of kPrefillRows rows; when they cannot fill the GPU, the key
-// axis is cut into chunks so that about two units land on every SM.
-Plan plan_prefill(int64_t m, int64_t n, int topk, int sms) {
+// Row blocks of kPrefillRows rows (4 with 64 heads); when they cannot fill
+// the GPU, the key axis is cut into chunks so that about two units land on
+// every SM.
+Plan plan_prefill(int64_t m, int64_t n, int topk, int sms, int H = kHeads) {
   Plan pl;
-  pl.R = kPrefillRows;
+  pl.H = H;
+  pl.R = H == 64 ? 4 : kPrefillRows;
+  pl.rows_per_unit = pl.R;
   const int64_t groups = ceil_div(m, pl.R);
   const int64_t axis = std::max<int64_t>(n, 1);
   pl.chunk_keys = static_cast<int>(round_up(axis, kBlockKeys));
@@ -264,9 +269,11 @@ Plan plan_prefill(int64_t m, int64_t n, int topk, int sms) {
 
 // One unit per (request, key chunk); chunks sized so that about four units
 // land on every SM (context lengths differ, so many chunks are short or empty).
-Plan plan_paged(int64_t B, int R, int max_blocks, int topk, int sms) {
+Plan plan_paged(int64_t B, int R, int max_blocks, int topk, int sms, int H = kHeads) {
   Plan pl;
-  pl.R = R;
+  pl.H = H;
+  pl.R = (H == 64 || R <= 4) ? 4 : 8;  // the kernel's rows; a request's R rows use the first R
+  pl.rows_per_unit = R;
   const int64_t axis = static_cast<int64_t>(max_blocks) * kPageSize;
   pl.chunk_keys = static_cast<int>(round_up(axis, kBlockKeys));
   pl.n_chunks = 1;
@@ -281,8 +288,15 @@ Plan plan_paged(int64_t B, int R, int max_blocks, int topk, int sms) {
 }
 
 int check_shape(int H, int D) {
-  if (H != kHeads || D != kDim)
-    return fail(FP8IDX_EUNSUPPORTED, "only H=32, D=128 are supported (got H=%d, D=%d)", H, D);
+  if ((H != 32 && H != 64) || D != kDim)
+    return fail(FP8IDX_EUNSUPPORTED, "only H=32 or 64 and D=128 are supported (got H=%d, D=%d)", H, D);
+  return FP8IDX_OK;
+}
+
+// Rows per request of the paged form: 1 to 8 (MTP verify widths), at most 4 with 64 heads.
+int check_rows_per_request(int R, int H) {
+  if (R < 1 || R > 8 || (H == 64 && R > 4))
+    return fail(FP8IDX_EUNSUPPORTED, "rows per request must be in [1, %d] with H=%d (got %d)", H == 64 ? 4 : 8, H, R);
   return FP8IDX_OK;
 }
 
@@ -381,10 +395,10 @@ int fp8idx_mqa_logits(const uint8_t* q, const uint8_t* k, const float* s, const 
 
   // One unit per 8-row block; small m splits the key axis (each unit writes
   // its own column range, so no merge is needed).
-  Plan pl = plan_prefill(m, n, 1, sms);
+  Plan pl = plan_prefill(m, n, 1, sms, H);
   IndexerParams p;
   memset(&p, 0, sizeof(p));
-  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, m * kHeads, pl.R * kHeads));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, m * H, pl.R * H));
   FP8IDX_TRY(make_rows128_map(&p.tmap_k, k, n, kBlockKeys));
   p.s = s;
   p.w = w;
@@ -392,6 +406,7 @@ int fp8idx_mqa_logits(const uint8_t* q, const uint8_t* k, const float* s, const 
   p.ke = ke;
   p.n = n;
   p.m = static_cast<int>(m);
+  p.rows_per_unit = pl.rows_per_unit;
   p.topk = 1;
   p.n_chunks = pl.n_chunks;
   p.chunk_keys = pl.chunk_keys;
@@ -406,7 +421,7 @@ int fp8idx_mqa_logits(const uint8_t* q, const uint8_t* k, const float* s, const 
   p.status = status;
   p.wait_limit_ns = g_wait_limit_ns;
   p.debug_withhold_first_tile = g_debug_withhold;
-  e = launch_indexer_prefill_logits(p, pl.grid, st);
+  e = launch_indexer_prefill_logits(p, H, pl.grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "mqa_logits launch");
   return ok();
 }
@@ -429,10 +444,10 @@ int fp8idx_topk_rows(const float* logits, int64_t ld, const int32_t* ks, const i
 }
 
 size_t fp8idx_mqa_logits_topk_workspace(int64_t m, int64_t n, int H, int D, int topk) {
-  if (H != kHeads || D != kDim || topk < 1 || topk > kMaxTopK || m < 0 || n < 0) return 0;
+  if ((H != 32 && H != 64) || D != kDim || topk < 1 || topk > kMaxTopK || m < 0 || n < 0) return 0;
   const int sms = device_sms();
   if (sms <= 0) return 0;
-  return plan_prefill(std::max<int64_t>(m, 1), n, topk, sms).total;
+  return plan_prefill(std::max<int64_t>(m, 1), n, topk, sms, H).total;
 }
 
 int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, const float* w,
@@ -447,7 +462,7 @@ int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, c
     return fail(FP8IDX_EINVAL, "out_idx must be non-null; outputs 4-byte aligned");
   const int sms = device_sms();
   if (sms <= 0) return fail(FP8IDX_ECUDA, "no CUDA device");
-  Plan pl = plan_prefill(m, n, topk, sms);
+  Plan pl = plan_prefill(m, n, topk, sms, H);
   if (!ws || !aligned(ws, 256)) return fail(FP8IDX_EINVAL, "workspace must be non-null and 256-byte aligned");
   if (ws_bytes < pl.total)
     return fail(FP8IDX_EWORKSPACE, "workspace too small (%zu < %zu bytes)", ws_bytes, pl.total);
@@ -462,7 +477,7 @@ int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, c
   }
   IndexerParams p;
   memset(&p, 0, sizeof(p));
-  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, m * kHeads, pl.R * kHeads));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, m * H, pl.R * H));
   FP8IDX_TRY(make_rows128_map(&p.tmap_k, k, n, kBlockKeys));
   p.s = s;
   p.w = w;
@@ -473,17 +488,17 @@ int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, c
   p.topk = topk;
   p.out_idx = out_idx;
   p.out_vals = out_vals;
-  return run_fused_topk(pl, p, wsb, false, pl.R, m, st);
+  return run_fused_topk(pl, p, wsb, false, m, st);
 }
 
 size_t fp8idx_paged_mqa_logits_topk_workspace(int64_t B, int R, int max_blocks, int H, int D,
                                               int topk) {
-  if (H != kHeads || D != kDim || topk < 1 || topk > kMaxTopK || B < 0 || max_blocks < 1 ||
-      (R != 4 && R != 8))
+  if ((H != 32 && H != 64) || D != kDim || topk < 1 || topk > kMaxTopK || B < 0 || max_blocks < 1 || R < 1 ||
+      R > 8 || (H == 64 && R > 4))
     return 0;
   const int sms = device_sms();
   if (sms <= 0) return 0;
-  return plan_paged(std::max<int64_t>(B, 1), R, max_blocks, topk, sms).total;
+  return plan_paged(std::max<int64_t>(B, 1), R, max_blocks, topk, sms, H).total;
 }
 
 int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const float* s_pages,
@@ -495,7 +510,7 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
   FP8IDX_TRY(check_shape(H, D));
   FP8IDX_TRY(check_topk(topk));
   if (page_size != kPageSize) return fail(FP8IDX_EUNSUPPORTED, "page_size must be 64 (got %d)", page_size);
-  if (R != 4 && R != 8) return fail(FP8IDX_EUNSUPPORTED, "rows per request must be 4 or 8 (got %d)", R);
+  FP8IDX_TRY(check_rows_per_request(R, H));
   if (B < 0 || num_pages < 0 || max_blocks < 1) return fail(FP8IDX_EINVAL, "bad sizes");
   if (B * R > (int64_t(1) << 25)) return fail(FP8IDX_EINVAL, "too many rows");
   if (static_cast<int64_t>(max_blocks) * kPageSize >= (int64_t(1) << 31) - kBlockKeys ||
@@ -512,7 +527,7 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
     return fail(FP8IDX_EINVAL, "pointers must be 4-byte aligned");
   const int sms = device_sms();
   if (sms <= 0) return fail(FP8IDX_ECUDA, "no CUDA device");
-  Plan pl = plan_paged(B, R, max_blocks, topk, sms);
+  Plan pl = plan_paged(B, R, max_blocks, topk, sms, H);
   if (!ws || !aligned(ws, 256)) return fail(FP8IDX_EINVAL, "workspace must be non-null and 256-byte aligned");
   if (ws_bytes < pl.total)
     return fail(FP8IDX_EWORKSPACE, "workspace too small (%zu < %zu bytes)", ws_bytes, pl.total);
@@ -527,7 +542,7 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
   }
   IndexerParams p;
   memset(&p, 0, sizeof(p));
-  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, B * R * kHeads, R * kHeads));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, B * R * H, pl.R * H));
   FP8IDX_TRY(make_rows128_map(&p.tmap_k, k_pages, num_pages * kPageSize, kPageSize));
   p.s = s_pages;
   p.w = w;
@@ -539,7 +554,7 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
   p.topk = topk;
   p.out_idx = out_idx;
   p.out_vals = out_vals;
-  return run_fused_topk(pl, p, wsb, true, R, B * R, st);
+  return run_fused_topk(pl, p, wsb, true, B * R, st);
 }
 
 // Allocation-free form of fp8idx_mqa_logits_topk for callers that cannot
@@ -574,7 +589,7 @@ int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const flo
   Plan pl;
   int g = sms;
   for (; g >= 1; --g) {
-    pl = plan_prefill(m, n, topk, g);
+    pl = plan_prefill(m, n, topk, g, H);
     if (pl.total <= kNoAllocScratchBytes) break;
   }
   if (g < 1)
@@ -590,7 +605,7 @@ int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const flo
   }
   IndexerParams p;
   memset(&p, 0, sizeof(p));
-  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, m * kHeads, pl.R * kHeads));
+  FP8IDX_TRY(make_rows128_map(&p.tmap_q, q, m * H, pl.R * H));
   FP8IDX_TRY(make_rows128_map(&p.tmap_k, k, n, kBlockKeys));
   p.s = s;
   p.w = w;
@@ -601,7 +616,7 @@ int fp8idx_mqa_logits_topk_noalloc(const uint8_t* q, const uint8_t* k, const flo
   p.topk = topk;
   p.out_idx = out_idx;
   p.out_vals = out_vals;
-  const int rc = run_fused_topk(pl, p, wsb, false, pl.R, m, st);
+  const int rc = run_fused_topk(pl, p, wsb, false, m, st);
   if (rc != FP8IDX_OK) return rc;
   return ok();
 }

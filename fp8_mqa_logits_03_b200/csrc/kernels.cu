@@ -48,10 +48,11 @@ namespace fp8idx {
 // four warps, one per TMEM lane quadrant (warp % 4), each warpgroup owning RW
 // rows of the unit.  More epilogue warpgroups with fewer rows each give every
 // SM sub-partition more independent warps to hide the epilogue's latencies.
-template <int R, bool PAGED>
+template <int R, bool PAGED, int H>
 struct Cfg {
-  static constexpr int N = R * kHeads;         // MMA N: (row, head) columns
+  static constexpr int N = R * H;              // MMA N: (row, head) columns
   static constexpr int RW = R == 8 ? 4 : 2;    // rows per epilogue warpgroup
+  static constexpr int NC = RW * H / 32;       // 32-column TMEM chunks per epilogue warp
   static constexpr int EWG = R / RW;           // epilogue warpgroups
   static constexpr int EPI_WARPS = 4 * EWG;
   static constexpr int THREADS = 32 * (4 + EPI_WARPS);
@@ -62,6 +63,7 @@ struct Cfg {
   static constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockKeys, N);
   static_assert(N <= 256 && N % 16 == 0, "MMA N out of range");
   static_assert(R % RW == 0 && EPI_WARPS <= kMaxEpiWarps, "epilogue layout");
+  static_assert(H % 32 == 0 && (NC == 2 || NC == 4), "32-column chunks per epilogue warp");
 };
 
 constexpr int kNB = 512;         // histogram bins per row
@@ -119,16 +121,16 @@ struct SmemLayout {
   int q, stage, bar, misc, w, rows, meta, hist, esel, ssel, up, at, total;
 };
 
-template <int R, bool PAGED>
+template <int R, bool PAGED, int H>
 __host__ __device__ constexpr SmemLayout smem_layout() {
-  using C = Cfg<R, PAGED>;
+  using C = Cfg<R, PAGED, H>;
   SmemLayout L{};
   L.q = 0;
   L.stage = C::Q_BYTES;
   L.bar = L.stage + C::STAGES * C::TILE_BYTES;
   L.misc = L.bar + 8 * (2 * C::STAGES + 20);
   L.w = L.misc + 64;
-  L.rows = L.w + R * kHeads * 4;
+  L.rows = L.w + R * H * 4;
   L.meta = L.rows + 2 * R * static_cast<int>(sizeof(RowState));
   L.hist = L.meta + 2 * static_cast<int>(sizeof(SlotMeta));
   L.esel = L.hist + 2 * R * kNB * 4;
@@ -158,8 +160,8 @@ __device__ __forceinline__ Unit get_unit(const IndexerParams& p, int u) {
   Unit U;
   const int grp = u / p.n_chunks;
   const int c = u - grp * p.n_chunks;
-  U.row0 = grp * R;
-  U.nrows = min(R, p.m - U.row0);
+  U.row0 = grp * p.rows_per_unit;  // (<= R: the MMA's row capacity; rows past nrows are idle)
+  U.nrows = min(p.rows_per_unit, p.m - U.row0);
   U.req = grp;
   U.len_clamped = false;
   int lo, hi, axis;
@@ -773,10 +775,10 @@ __device__ __forceinline__ int estimate_target(int k, int seen, int vtot) {
 
 // ------------------------------------------------------------------ kernel
 
-template <int R, bool PAGED, int MODE>
-__global__ void __launch_bounds__(Cfg<R, PAGED>::THREADS, 1) indexer_kernel(const __grid_constant__ IndexerParams p) {
-  using C = Cfg<R, PAGED>;
-  constexpr SmemLayout SL = smem_layout<R, PAGED>();
+template <int R, bool PAGED, int H, int MODE>
+__global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(const __grid_constant__ IndexerParams p) {
+  using C = Cfg<R, PAGED, H>;
+  constexpr SmemLayout SL = smem_layout<R, PAGED, H>();
   constexpr int N = C::N;
   constexpr int RW = C::RW;
   constexpr int S = C::STAGES;
@@ -897,7 +899,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED>::THREADS, 1) indexer_kernel(cons
         if (!wait_phase<kProd>(qempty, qphase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
         qphase ^= 1;
         mbar_arrive_expect_tx(qfull, C::Q_BYTES);
-        tma_load_2d(q_smem, &p.tmap_q, qfull, 0, U.row0 * kHeads);
+        tma_load_2d(q_smem, &p.tmap_q, qfull, 0, U.row0 * H);
         const int32_t* bt = PAGED ? p.block_table + static_cast<int64_t>(U.req) * p.max_blocks : nullptr;
         for (int t = 0; t < U.ntiles; ++t) {
           if (!wait_phase<kProd>(&empty[stage], phase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
@@ -994,7 +996,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED>::THREADS, 1) indexer_kernel(cons
     const int qd = warp & 3;  // TMEM lane quadrant == key block of 32 == buffer segment
     const int tid_wg = qd * 32 + lane;
     const int bar_id = 1 + g;
-    float* ws_g = w_smem + g * RW * kHeads;
+    float* ws_g = w_smem + g * RW * H;
     Group<1> grp{esel_smem + ew * kSelWords, nullptr, esel_smem + ew * kSelWords + 256, 0, lane};
     const int k = p.topk;
     const int cap = p.cand_cap;
@@ -1071,7 +1073,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED>::THREADS, 1) indexer_kernel(cons
             lo = max(__ldg(p.ks + row), 0);
             hi = max(lo, min(__ldg(p.ke + row), static_cast<int>(p.n)));
           } else {
-            const int e = U.len - R + rl + 1;
+            const int e = U.len - p.rows_per_unit + rl + 1;
             hi = max(min(e, U.len), 0);
           }
           vtot = hi - lo;
@@ -1083,9 +1085,9 @@ __global__ void __launch_bounds__(Cfg<R, PAGED>::THREADS, 1) indexer_kernel(cons
         rs[tid_wg].hi = hi;
         rs[tid_wg].vtot = vtot;
       }
-      if (tid_wg < RW * kHeads) {
-        const int rl = g * RW + tid_wg / kHeads;
-        ws_g[tid_wg] = rl < U.nrows ? __ldg(p.w + static_cast<int64_t>(U.row0 + rl) * kHeads + tid_wg % kHeads) : 0.f;
+      for (int x = tid_wg; x < RW * H; x += 128) {
+        const int rl = g * RW + x / H;
+        ws_g[x] = rl < U.nrows ? __ldg(p.w + static_cast<int64_t>(U.row0 + rl) * H + x % H) : 0.f;
       }
       if (MODE == kModeTopK) {
         if (tid_wg < RW) {
@@ -1161,37 +1163,46 @@ __global__ void __launch_bounds__(Cfg<R, PAGED>::THREADS, 1) indexer_kernel(cons
         const uint32_t a = T & 1, aph = (T >> 1) & 1;
         if (!wait_phase<kSpin>(&tfull[a], aph, abort_flag, p.status, limit)) aborted = true;
         tc_fence_after();
-        // Rows in pairs (64 TMEM columns per pair); the next pair's loads are
-        // in flight while the current pair's sums are formed.  The last wait
-        // leaves the whole accumulator in registers: release it to the MMA.
-        // (fma with +0: an exactly zero head sum gives +0 whatever the sign
-        // of the scale.)
-        static_assert(RW == 2 || RW == 4, "rows per warpgroup");
-        float L[RW];
+        // The warp's RW rows are NC chunks of 32 TMEM columns (chunk c at
+        // column g * RW * H + 32 c, its head weights at ws_g + 32 c), taken in
+        // pairs; the next pair's loads are in flight while the current pair's
+        // sums are formed.  The last wait leaves the whole accumulator in
+        // registers: release it to the MMA.  A row's logit sums its H / 32
+        // chunks.  (fma with +0: an exactly zero head sum gives +0 whatever
+        // the sign of the scale.)
+        constexpr int NC = C::NC;
+        float Lc[NC];
         {
+          const uint32_t col0 = lane_addr + a * N + g * RW * H;
           uint32_t xa[32], xb[32];
-          tmem_ld32(lane_addr + a * N + (g * RW + 0) * kHeads, xa);
-          tmem_ld32(lane_addr + a * N + (g * RW + 1) * kHeads, xb);
+          tmem_ld32(col0, xa);
+          tmem_ld32(col0 + 32, xb);
           tmem_ld_wait();
-          if (RW == 2) {
+          if (NC == 2) {
             tc_fence_before();
             __syncwarp();
             mbar_arrive_if(lane == 0, &tempty[a]);
-            relu_dot32_x2_pair(xa, xb, ws_g, ws_g + kHeads, L[0], L[1]);
+            relu_dot32_x2_pair(xa, xb, ws_g, ws_g + 32, Lc[0], Lc[1]);
           } else {
             uint32_t xc[32], xd[32];
-            tmem_ld32(lane_addr + a * N + (g * RW + 2) * kHeads, xc);
-            tmem_ld32(lane_addr + a * N + (g * RW + 3) * kHeads, xd);
-            relu_dot32_x2_pair(xa, xb, ws_g, ws_g + kHeads, L[0], L[1]);
+            tmem_ld32(col0 + 64, xc);
+            tmem_ld32(col0 + 96, xd);
+            relu_dot32_x2_pair(xa, xb, ws_g, ws_g + 32, Lc[0], Lc[1]);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             mbar_arrive_if(lane == 0, &tempty[a]);
-            relu_dot32_x2_pair(xc, xd, ws_g + 2 * kHeads, ws_g + 3 * kHeads, L[2], L[RW - 1]);
+            relu_dot32_x2_pair(xc, xd, ws_g + 64, ws_g + 96, Lc[2], Lc[NC - 1]);
           }
         }
+        float L[RW];
 #pragma unroll
-        for (int r = 0; r < RW; ++r) L[r] = fmaf(L[r], sj, 0.f);
+        for (int r = 0; r < RW; ++r) {
+          float acc = Lc[r * (H / 32)];
+#pragma unroll
+          for (int c = 1; c < H / 32; ++c) acc += Lc[r * (H / 32) + c];
+          L[r] = fmaf(acc, sj, 0.f);
+        }
 
         if (MODE == kModeLogits) {
 #pragma unroll
@@ -1402,9 +1413,9 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
   const int unit_row = row / p.R;  // row block / request
   const int rl = row - unit_row * p.R;
   const size_t u0 = static_cast<size_t>(unit_row) * p.n_chunks;
-  const uint2* base = p.part + (u0 * p.R + rl) * p.topk;
-  const size_t stride = static_cast<size_t>(p.R) * p.topk;
-  const int* cnt = p.part_cnt + u0 * p.R + rl;
+  const uint2* base = p.part + (u0 * p.R_part + rl) * p.topk;
+  const size_t stride = static_cast<size_t>(p.R_part) * p.topk;
+  const int* cnt = p.part_cnt + u0 * p.R_part + rl;
   Group<kMergeWarps> g{hist, red, &counter, 1, static_cast<int>(threadIdx.x)};
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int total = -1;  // pairs surviving in all chunks (-1: not scanned)
@@ -1412,7 +1423,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
     const int c = threadIdx.x;
     // a count outside [0, topk] only follows an aborted indexer launch (the
     // device status says so); clamped, it still keeps every access in bounds
-    const int v = c < p.n_chunks ? min(max(__ldg(cnt + static_cast<size_t>(c) * p.R), 0), p.topk) : 0;
+    const int v = c < p.n_chunks ? min(max(__ldg(cnt + static_cast<size_t>(c) * p.R_part), 0), p.topk) : 0;
     int incl = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -1448,7 +1459,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
     const SelectResult sel = group_select<kMergeWarps>(src, total, p.topk, g);
     nout = group_emit<kMergeWarps>(src, total, sel, g, emit);
   } else {
-    const PartSrc src{base, cnt, stride, p.R, p.topk};
+    const PartSrc src{base, cnt, stride, p.R_part, p.topk};
     const int all = p.n_chunks * p.topk;
     const SelectResult sel = group_select<kMergeWarps>(src, all, p.topk, g);
     nout = group_emit<kMergeWarps>(src, all, sel, g, emit);
@@ -1519,26 +1530,31 @@ __global__ void fill_empty_kernel(int32_t* out_idx, float* out_vals, int64_t tot
 
 // ------------------------------------------------------------------ launchers
 
-template <int R, bool PAGED, int MODE>
+template <int R, bool PAGED, int H, int MODE>
 static cudaError_t launch_indexer(const IndexerParams& p, int grid, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(smem_layout<R, PAGED>().total) + 1024;
-  auto kern = indexer_kernel<R, PAGED, MODE>;
+  const size_t smem = static_cast<size_t>(smem_layout<R, PAGED, H>().total) + 1024;
+  auto kern = indexer_kernel<R, PAGED, H, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, Cfg<R, PAGED>::THREADS, smem, st>>>(p);
+  kern<<<grid, Cfg<R, PAGED, H>::THREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_indexer_prefill_logits(const IndexerParams& p, int grid, cudaStream_t st) {
-  return launch_indexer<kPrefillRows, false, kModeLogits>(p, grid, st);
+// Instantiations: 32 heads with 8-row prefill units (4- or 8-row paged
+// units); 64 heads with 4-row units (N = 4 x 64 = 256 columns).
+cudaError_t launch_indexer_prefill_logits(const IndexerParams& p, int H, int grid, cudaStream_t st) {
+  if (H == 64) return launch_indexer<4, false, 64, kModeLogits>(p, grid, st);
+  return launch_indexer<kPrefillRows, false, 32, kModeLogits>(p, grid, st);
 }
-cudaError_t launch_indexer_prefill_topk(const IndexerParams& p, int grid, cudaStream_t st) {
-  return launch_indexer<kPrefillRows, false, kModeTopK>(p, grid, st);
+cudaError_t launch_indexer_prefill_topk(const IndexerParams& p, int H, int grid, cudaStream_t st) {
+  if (H == 64) return launch_indexer<4, false, 64, kModeTopK>(p, grid, st);
+  return launch_indexer<kPrefillRows, false, 32, kModeTopK>(p, grid, st);
 }
-cudaError_t launch_indexer_paged_topk(const IndexerParams& p, int R, int grid, cudaStream_t st) {
-  if (R == 8) return launch_indexer<8, true, kModeTopK>(p, grid, st);
-  return launch_indexer<4, true, kModeTopK>(p, grid, st);
+cudaError_t launch_indexer_paged_topk(const IndexerParams& p, int R, int H, int grid, cudaStream_t st) {
+  if (H == 64) return launch_indexer<4, true, 64, kModeTopK>(p, grid, st);
+  if (R == 8) return launch_indexer<8, true, 32, kModeTopK>(p, grid, st);
+  return launch_indexer<4, true, 32, kModeTopK>(p, grid, st);
 }
 
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t st) {

@@ -57,6 +57,7 @@ struct IndexerParams {
   int max_blocks;
   int num_pages;
   int topk;
+  int rows_per_unit;  // query rows of a row block / request (at most the kernel's row capacity)
   int n_chunks;     // key chunks per row block / request
   int chunk_keys;   // keys per chunk (multiple of 128)
   int num_units;    // row blocks (or requests) x n_chunks
@@ -90,7 +91,8 @@ struct MergeParams {
   const uint2* part;
   const int* part_cnt;
   int rows;          // total query rows
-  int R;             // rows per unit
+  int R;             // query rows per row block / request
+  int R_part;        // row stride of the partial lists (the kernel's row capacity)
   int n_chunks;
   int topk;
   int32_t* out_idx;
@@ -113,9 +115,9 @@ struct TopkRowsParams {
 };
 
 // Launchers (kernels.cu).  They only enqueue work; validation is the caller's.
-cudaError_t launch_indexer_prefill_logits(const IndexerParams& p, int grid, cudaStream_t st);
-cudaError_t launch_indexer_prefill_topk(const IndexerParams& p, int grid, cudaStream_t st);
-cudaError_t launch_indexer_paged_topk(const IndexerParams& p, int R, int grid, cudaStream_t st);
+cudaError_t launch_indexer_prefill_logits(const IndexerParams& p, int H, int grid, cudaStream_t st);
+cudaError_t launch_indexer_prefill_topk(const IndexerParams& p, int H, int grid, cudaStream_t st);
+cudaError_t launch_indexer_paged_topk(const IndexerParams& p, int R, int H, int grid, cudaStream_t st);
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t st);
 cudaError_t launch_topk_rows(const TopkRowsParams& p, cudaStream_t st);
 cudaError_t launch_fill_empty(int32_t* out_idx, float* out_vals, int rows, int topk,

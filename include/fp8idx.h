@@ -16,7 +16,7 @@
  *
  * q and k are fp8 e4m3fn bytes (the "e4m3fn" format named on the
  * "Serve GLM-5.3-Flash on SM80" page, commit notes); s and w are fp32; ks
- * and ke are int32.  H must be 32 and D must be 128.
+ * and ke are int32.  H is 32 (the pages' index_n_heads) or 64; D is 128.
  *
  * Conventions shared by every call:
  *   - All data pointers are DEVICE pointers owned by the caller.  The library
@@ -30,8 +30,9 @@
  *     workspaces 256 bytes.
  *   - Errors are reported before anything is launched and leave the outputs
  *     untouched: FP8IDX_EINVAL (null pointer, misalignment, negative size,
- *     topk outside [1, 2048], ld_logits < n), FP8IDX_EUNSUPPORTED (H != 32,
- *     D != 128, page_size != 64, rows_per_request not 4 or 8),
+ *     topk outside [1, 2048], ld_logits < n), FP8IDX_EUNSUPPORTED (H not 32
+ *     or 64, D != 128, page_size != 64, rows per request outside [1, 8], or
+ *     above 4 with H = 64),
  *     FP8IDX_EWORKSPACE (workspace smaller than the *_workspace() size),
  *     FP8IDX_ECUDA (a CUDA call failed; see fp8idx_last_error()).
  *     m == 0 (or B == 0) is a no-op returning FP8IDX_OK.
@@ -124,7 +125,8 @@ int fp8idx_mqa_logits_topk(const uint8_t* q, const uint8_t* k, const float* s, c
  *   block_table [B, max_blocks] int32 (entries past a request's pages are
  *               never read)                   seq_lens [B] int32
  *   out_idx     [B * R, topk] int32           out_vals [B * R, topk] fp32 or NULL
- * R must be 4 or 8; page_size must be 64.
+ * R is 1 (decode) to 8 (MTP verify widths; the megakernels page names
+ * q4-q8), at most 4 with H = 64; page_size must be 64.
  */
 size_t fp8idx_paged_mqa_logits_topk_workspace(int64_t B, int R, int max_blocks, int H, int D,
                                               int topk);

@@ -69,9 +69,11 @@ def test_paged_rejects(L):
         return L.fp8idx_paged_mqa_logits_topk(q, FAKE, FAKE, FAKE, FAKE, FAKE, B, R, max_blocks,
                                               num_pages, page_size, H, 128, topk, FAKE, None, FAKE,
                                               1 << 20, None)
-    assert call(R=3) == fx.EUNSUPPORTED
+    assert call(R=0) == fx.EUNSUPPORTED
+    assert call(R=9) == fx.EUNSUPPORTED
     assert call(page_size=32) == fx.EUNSUPPORTED
-    assert call(H=64) == fx.EUNSUPPORTED
+    assert call(H=48) == fx.EUNSUPPORTED
+    assert call(H=64, R=5) == fx.EUNSUPPORTED    # 64 heads: at most 4 rows per request
     assert call(max_blocks=0) == fx.EINVAL
     assert call(q=MIS) == fx.EINVAL
     assert call(B=0) == fx.OK
@@ -79,7 +81,9 @@ def test_paged_rejects(L):
 
 def test_workspace_queries_reject_bad_shapes(L):
     assert L.fp8idx_mqa_logits_topk_workspace(8, 100, 32, 128, 0) == 0
-    assert L.fp8idx_paged_mqa_logits_topk_workspace(4, 3, 16, 32, 128, 2048) == 0
+    assert L.fp8idx_paged_mqa_logits_topk_workspace(4, 9, 16, 32, 128, 2048) == 0
+    assert L.fp8idx_paged_mqa_logits_topk_workspace(4, 5, 16, 64, 128, 2048) == 0
+    assert L.fp8idx_mqa_logits_topk_workspace(8, 100, 48, 128, 16) == 0
 
 
 def test_act_quant_store_rejects(L):
