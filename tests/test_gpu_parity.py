@@ -296,3 +296,57 @@ def test_paged_estimate_rejected_and_repaired():
     assert stats["status"] == 0
     assert stats["repairs"] > 0, stats
     _paged_check(d, idx.cpu().numpy(), vals.cpu().numpy(), np.arange(len(lengths) * R), k)
+
+
+# ---------------------------------------------------------------------------- wide samples, full rows
+
+def _blocks_and_random(m, count, seed, block=8):
+    """The first and last row blocks plus `count` random rows."""
+    g = np.random.default_rng(seed)
+    rows = set(range(min(block, m))) | set(range(max(0, m - block), m))
+    rows.update(g.choice(m, size=min(count, m), replace=False).tolist())
+    return np.array(sorted(rows))
+
+
+def test_cp_slice_210k_fused_and_chained_sampled():
+    """Workload 3 (7500 rows over 210000 keys): the fused call and the chained
+    path (logits in row chunks of at most 2 GiB, then topk_rows on each chunk,
+    the loop of the chunking benchmark) on the first and last row blocks and
+    256 random rows, against one oracle evaluation."""
+    d = workloads.make_workload(3)
+    m, n, k = d["m"], d["n"], workloads.TOPK
+    idx, vals = _fused_call(d, k)
+    t = _to(d)
+    rows_per_chunk = max(1, (2 << 30) // (4 * n))
+    chained = torch.empty((m, k), dtype=torch.int32, device="cuda")
+    logits = torch.empty((rows_per_chunk, n), dtype=torch.float32, device="cuda")
+    for r0 in range(0, m, rows_per_chunk):
+        r1 = min(m, r0 + rows_per_chunk)
+        lg = logits[: r1 - r0]
+        fx.mqa_logits(t["q"][r0:r1], t["k"], t["s"], t["w"][r0:r1], t["ks"][r0:r1], t["ke"][r0:r1], logits=lg)
+        fx.topk_rows(lg, t["ks"][r0:r1], t["ke"][r0:r1], k, out=chained[r0:r1])
+    torch.cuda.synchronize()
+    assert fx.read_device_status(None) == 0
+    rows = _blocks_and_random(m, 256, 3)
+    ref = _oracle_rows(d, rows)
+    fi, fv, ci = idx.cpu().numpy(), vals.cpu().numpy(), chained.cpu().numpy()
+    for r, i in enumerate(rows):
+        lo, hi = row_range(d["ks"][i], d["ke"][i], n)
+        check_topk_row(fi[i], ref[r], lo, hi, k, fv[i], f"fused row {i}")
+        check_topk_row(ci[i], ref[r], lo, hi, k, None, f"chained row {i}")
+
+
+def test_causal_prefill_all_rows():
+    """Workload 1 (8192 rows over 35000 keys), every row against the oracle."""
+    d = workloads.make_workload(1)
+    m, n, k = d["m"], d["n"], workloads.TOPK
+    idx, vals = _fused_call(d, k)
+    fi, fv = idx.cpu().numpy(), vals.cpu().numpy()
+    diffs = 0
+    for r0 in range(0, m, 512):
+        rows = np.arange(r0, min(m, r0 + 512))
+        ref = _oracle_rows(d, rows)
+        for r, i in enumerate(rows):
+            lo, hi = row_range(d["ks"][i], d["ke"][i], n)
+            diffs += check_topk_row(fi[i], ref[r], lo, hi, k, fv[i], f"row {i}")
+    print(f"all {m} rows match; {diffs} keys swapped inside the tie band")
