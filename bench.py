@@ -343,7 +343,7 @@ def make_case(fx, index, dev, path="fused"):
 
         def call():
             fx.paged_mqa_logits_topk(**dv, R=R, topk=topk, out=out, workspace=ws)
-        kernel = "indexer_kernel<4,true,1> (paged fused logits + top-k) + merge_kernel"
+        kernel = "indexer_kernel<4,true,32,1> (paged fused logits + top-k) + merge_kernel + repair launch"
         bound = "hbm"
     else:
         keys = ("q", "k", "s", "w", "ks", "ke")
@@ -357,7 +357,7 @@ def make_case(fx, index, dev, path="fused"):
 
         def call():
             fx.mqa_logits_topk(**dv, topk=topk, out=out, workspace=ws)
-        kernel = "indexer_kernel<8,false,1> (fused logits + top-k)"
+        kernel = "indexer_kernel<8,false,32,1> (fused logits + top-k) + repair launch"
         bound = "tensor"
         if path == "chained":
             m, n = d["m"], d["n"]
@@ -377,7 +377,9 @@ def make_case(fx, index, dev, path="fused"):
             launches = 2 * len(chunks)
     out_host = torch.empty(out.shape, dtype=torch.int32).pin_memory()
     if path == "fused":
-        launches = 2 if index in (0, 4) else 1  # + the merge kernel when the key axis is split
+        # the indexer, the merge when the key axis is split, and the repair launch
+        # (which ends at once when no estimated threshold was rejected)
+        launches = 3 if index in (0, 4) else 2
     return dict(d=d, call=call, host=host, dv=dv, out=out, out_host=out_host, ws=ws, pairs=pairs,
                 flops=FLOP_PER_PAIR * pairs, bytes=nbytes, kernel=kernel, bound=bound,
                 launches=launches, metric=METRIC, unit=UNIT)
@@ -424,6 +426,90 @@ def roofline_of(case, mean_s, peaks):
 
 
 SUITE = [(0, "fused"), (2, "fused"), (3, "fused"), (4, "fused"), (4, "act_quant")]
+
+# Index preparation at the shape of the "reuse inference metadata" page: 8
+# requests of 1M tokens, 1 (decode), 4 (MTP verify) or 16 (prefill chunk)
+# query rows each; a step prepares the rows' key ranges and maps every row's
+# top-2048 positions to KV slots through the token table.  The page's H200
+# figures after its change are quoted as context.
+INDEX_PREP = [("decode", 1, 1.77), ("mtp4", 4, 1.81), ("prefill16", 16, 3.63)]
+
+
+def time_graph(call, reps_target_ms=200.0, samples=3):
+    """Median over `samples` of the mean replay time (us) of a CUDA graph of
+    `call`, each sample replaying for about reps_target_ms."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            call()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(20):
+        g.replay()
+    e1.record()
+    e1.synchronize()
+    per = max(e0.elapsed_time(e1) / 20, 1e-4)
+    reps = max(20, int(reps_target_ms / per))
+    out = []
+    for _ in range(samples):
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        e1.synchronize()
+        out.append(e0.elapsed_time(e1) / reps * 1e3)
+    del g
+    return statistics.median(out)
+
+
+def run_index_prep(fx, dev, B=8, L=1 << 20, topk=workloads.TOPK, seed=20270):
+    """Index preparation + top-k transform at 8 x 1M tokens (CUDA-graph
+    replays), and the parallel long-context ragged copy."""
+    gen = torch.Generator().manual_seed(seed)
+    table_rows = B + 1
+    table = torch.randint(0, 1 << 30, (table_rows, L), generator=gen, dtype=torch.int32).to(dev)
+    seq = torch.full((B,), L, dtype=torch.int32, device=dev)
+    req = torch.arange(B, dtype=torch.int32, device=dev)
+    res = {}
+    for name, qn, h200_us in INDEX_PREP:
+        rows = B * qn
+        q_len = torch.full((B,), qn, dtype=torch.int32, device=dev)
+        ks = torch.empty(rows, dtype=torch.int32, device=dev)
+        ke = torch.empty_like(ks)
+        rt = torch.empty_like(ks)
+        # top-k positions inside each row's request segment (ragged key space)
+        base = (torch.arange(rows, device=dev) // qn).to(torch.int64) * L
+        pos = (torch.randint(0, L - qn, (rows, topk), generator=gen).to(dev) + base[:, None]).to(torch.int32)
+        out = torch.empty_like(pos)
+
+        def step():
+            fx.prepare_ragged(seq, q_len, req, table, q_cap=rows, with_ragged=False, ks=ks, ke=ke, row_table=rt)
+            fx.topk_transform(pos, table, 1, row_base=ks, row_table=rt, out=out)
+        us = time_graph(step)
+        res[name] = {"us_per_step": us, "rows": rows, "topk": topk, "requests": B, "tokens_per_request": L,
+                     "launches": 2, "page_h200_us_context": h200_us}
+    # the ragged index copy of the whole batch (8M token slots), read + write
+    q1 = torch.ones(B, dtype=torch.int32, device=dev)
+    ragged = torch.empty(B * L, dtype=torch.int32, device=dev)
+    ks = torch.empty(B, dtype=torch.int32, device=dev)
+    ke, rt = torch.empty_like(ks), torch.empty_like(ks)
+
+    def copy():
+        fx.prepare_ragged(seq, q1, req, table, q_cap=B, ragged=ragged, ks=ks, ke=ke, row_table=rt)
+    us = time_graph(copy, reps_target_ms=100.0)
+    res["ragged_copy_8x1M"] = {"us_per_step": us, "gbs": 2 * 4 * B * L / (us * 1e-6) / 1e9,
+                              "bytes_per_step": 2 * 4 * B * L}
+    del table, ragged
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_suite(fx, dev, flush, stream, peaks, steps=10, warmup=3):
@@ -524,6 +610,7 @@ def run_ours(args, rank, world, local, pg):
         torch.cuda.empty_cache()
         fp8_meas = measure_fp8_peak(dev)
         suite = run_suite(fx, dev, flush, stream, load_peaks() + (fp8_meas,))
+        suite["index_prep_8x1M"] = run_index_prep(fx, dev)
         barrier(pg)
     if rank != 0:
         return None

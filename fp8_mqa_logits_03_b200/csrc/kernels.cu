@@ -56,7 +56,8 @@ struct Cfg {
   static constexpr int EWG = R / RW;           // epilogue warpgroups
   static constexpr int EPI_WARPS = 4 * EWG;
   static constexpr int THREADS = 32 * (4 + EPI_WARPS);
-  static constexpr int STAGES = PAGED ? (R == 8 ? 5 : 7) : 5;  // key-tile ring depth
+  // key-tile ring depth: what shared memory leaves next to two q blocks
+  static constexpr int STAGES = R == 8 ? 4 : (H == 64 ? 5 : (PAGED ? 7 : 5));
   static constexpr int Q_BYTES = N * kDim;
   static constexpr int TILE_BYTES = kBlockKeys * kDim;
   static constexpr int TMEM_COLS = 2 * N <= 256 ? 256 : 512;  // double-buffered accumulators
@@ -125,10 +126,10 @@ template <int R, bool PAGED, int H>
 __host__ __device__ constexpr SmemLayout smem_layout() {
   using C = Cfg<R, PAGED, H>;
   SmemLayout L{};
-  L.q = 0;
-  L.stage = C::Q_BYTES;
+  L.q = 0;  // two q blocks: the next unit's loads while this unit's MMAs run
+  L.stage = 2 * C::Q_BYTES;
   L.bar = L.stage + C::STAGES * C::TILE_BYTES;
-  L.misc = L.bar + 8 * (2 * C::STAGES + 20);
+  L.misc = L.bar + 8 * (2 * C::STAGES + 22);
   L.w = L.misc + 64;
   L.rows = L.w + R * H * 4;
   L.meta = L.rows + 2 * R * static_cast<int>(sizeof(RowState));
@@ -796,13 +797,13 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
   uint64_t* empty = bars + S;
   uint64_t* tfull = bars + 2 * S;
   uint64_t* tempty = bars + 2 * S + 2;
-  uint64_t* qfull = bars + 2 * S + 4;
-  uint64_t* qempty = bars + 2 * S + 5;
-  uint64_t* drain = bars + 2 * S + 6;
-  uint64_t* slot_full = bars + 2 * S + 7;
-  uint64_t* slot_empty = bars + 2 * S + 9;
-  uint64_t* uq_full = bars + 2 * S + 11;   // unit queue, 4 entries
-  uint64_t* uq_empty = bars + 2 * S + 15;
+  uint64_t* qfull = bars + 2 * S + 4;      // two q slots
+  uint64_t* qempty = bars + 2 * S + 6;
+  uint64_t* drain = bars + 2 * S + 8;
+  uint64_t* slot_full = bars + 2 * S + 9;
+  uint64_t* slot_empty = bars + 2 * S + 11;
+  uint64_t* uq_full = bars + 2 * S + 13;   // unit queue, 4 entries
+  uint64_t* uq_empty = bars + 2 * S + 17;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SL.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL.misc + 4);
   volatile int* uq = reinterpret_cast<volatile int*>(smem + SL.misc + 16);  // unit queue
@@ -837,8 +838,10 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
       mbar_init(&uq_full[x], 1);
       mbar_init(&uq_empty[x], 1 + C::EPI_WARPS);  // the MMA thread and every epilogue warp
     }
-    mbar_init(qfull, 1);
-    mbar_init(qempty, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&qfull[x], 1);
+      mbar_init(&qempty[x], 1);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -859,7 +862,8 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
       tma_prefetch_desc(&p.tmap_q);
       tma_prefetch_desc(&p.tmap_k);
       int stage = 0;
-      uint32_t phase = 0, qphase = 0;
+      uint32_t phase = 0;
+      int nq = 0;  // units with tiles so far: unit nq uses q slot nq & 1
       uint32_t issued_phase[S];
       bool issued[S];
 #pragma unroll
@@ -896,10 +900,11 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
         if (u < 0) break;
         const Unit U = get_unit<R, PAGED>(p, u);
         if (U.ntiles == 0) continue;
-        if (!wait_phase<kProd>(qempty, qphase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
-        qphase ^= 1;
-        mbar_arrive_expect_tx(qfull, C::Q_BYTES);
-        tma_load_2d(q_smem, &p.tmap_q, qfull, 0, U.row0 * H);
+        const int qs2 = nq & 1;
+        if (!wait_phase<kProd>(&qempty[qs2], ((nq >> 1) & 1) ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
+        ++nq;
+        mbar_arrive_expect_tx(&qfull[qs2], C::Q_BYTES);
+        tma_load_2d(q_smem + qs2 * C::Q_BYTES, &p.tmap_q, &qfull[qs2], 0, U.row0 * H);
         const int32_t* bt = PAGED ? p.block_table + static_cast<int64_t>(U.req) * p.max_blocks : nullptr;
         for (int t = 0; t < U.ntiles; ++t) {
           if (!wait_phase<kProd>(&empty[stage], phase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
@@ -944,7 +949,8 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, qphase = 0;
+      uint32_t phase = 0;
+      int nq = 0;  // units with tiles so far (the producer's q slot order)
       uint32_t T = 0;
       bool ok = true;
       bool any = false;
@@ -957,10 +963,11 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
         if (u < 0) break;
         const Unit U = get_unit<R, PAGED>(p, u);
         if (U.ntiles == 0) continue;
-        if (!wait_phase<kNap>(qfull, qphase, abort_flag, p.status, limit)) { ok = false; break; }
-        qphase ^= 1;
+        const int qs2 = nq & 1;
+        if (!wait_phase<kNap>(&qfull[qs2], (nq >> 1) & 1, abort_flag, p.status, limit)) { ok = false; break; }
+        ++nq;
         tc_fence_after();
-        const uint64_t bdesc = smem_desc_k128_sw128(q_addr);
+        const uint64_t bdesc = smem_desc_k128_sw128(q_addr + qs2 * C::Q_BYTES);
         for (int t = 0; t < U.ntiles; ++t, ++T) {
           const uint32_t a = T & 1, aph = (T >> 1) & 1;
           if (!wait_phase<kNap>(&tempty[a], aph ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
@@ -980,7 +987,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
             phase ^= 1;
           }
         }
-        if (ok) mma_commit(qempty);
+        if (ok) mma_commit(&qempty[qs2]);
       }
       if (any) {  // all MMAs retired before TMEM is released
         mma_commit(drain);
@@ -1156,28 +1163,41 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
       };
       float s_next = U.ntiles ? scale_of(key0) : 0.f;
       int next_vote = vote_interval(0) - 1;  // the same tile sequence in every warp
+      // The warp's RW rows are NC chunks of 32 TMEM columns (chunk c at column
+      // g * RW * H + 32 c, its head weights at ws_g + 32 c), taken in pairs; a
+      // later pair's loads are in flight while the pair before it is summed.
+      // With a single pair (NC == 2), the next tile's pair is loaded as soon
+      // as its accumulator is ready, before this tile's filter runs (xa, xb
+      // carry it from one iteration to the next); with two pairs the
+      // registers this would hold across the filter are not there.
+      constexpr bool kCarry = C::NC == 2;
+      uint32_t xa[32], xb[32];
+      if (kCarry && U.ntiles > 0) {
+        if (!wait_phase<kSpin>(&tfull[T & 1], (T >> 1) & 1, abort_flag, p.status, limit)) aborted = true;
+        tc_fence_after();
+        const uint32_t col0 = lane_addr + (T & 1) * N + g * RW * H;
+        tmem_ld32(col0, xa);
+        tmem_ld32(col0 + 32, xb);
+      }
       for (int t = 0; t < U.ntiles; ++t, ++T) {
         const int j = key0 + t * kBlockKeys;
         const float sj = 0.5f * s_next;  // relu_dot32_x2 returns twice the head sum
         s_next = scale_of(j + kBlockKeys);  // (0 past the end)
-        const uint32_t a = T & 1, aph = (T >> 1) & 1;
-        if (!wait_phase<kSpin>(&tfull[a], aph, abort_flag, p.status, limit)) aborted = true;
-        tc_fence_after();
-        // The warp's RW rows are NC chunks of 32 TMEM columns (chunk c at
-        // column g * RW * H + 32 c, its head weights at ws_g + 32 c), taken in
-        // pairs; the next pair's loads are in flight while the current pair's
-        // sums are formed.  The last wait leaves the whole accumulator in
-        // registers: release it to the MMA.  A row's logit sums its H / 32
-        // chunks.  (fma with +0: an exactly zero head sum gives +0 whatever
-        // the sign of the scale.)
+        const uint32_t a = T & 1;
+        // The last wait leaves the whole accumulator in registers: release it
+        // to the MMA.  A row's logit sums its H / 32 chunks.  (fma with +0: an
+        // exactly zero head sum gives +0 whatever the sign of the scale.)
         constexpr int NC = C::NC;
         float Lc[NC];
         {
           const uint32_t col0 = lane_addr + a * N + g * RW * H;
-          uint32_t xa[32], xb[32];
-          tmem_ld32(col0, xa);
-          tmem_ld32(col0 + 32, xb);
-          tmem_ld_wait();
+          if (!kCarry) {
+            if (!wait_phase<kSpin>(&tfull[a], (T >> 1) & 1, abort_flag, p.status, limit)) aborted = true;
+            tc_fence_after();
+            tmem_ld32(col0, xa);
+            tmem_ld32(col0 + 32, xb);
+          }
+          tmem_ld_wait();  // the first pair
           if (NC == 2) {
             tc_fence_before();
             __syncwarp();
@@ -1202,6 +1222,14 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
 #pragma unroll
           for (int c = 1; c < H / 32; ++c) acc += Lc[r * (H / 32) + c];
           L[r] = fmaf(acc, sj, 0.f);
+        }
+        if (kCarry && t + 1 < U.ntiles) {  // the next tile's pair, in flight during this tile's filter
+          const uint32_t an = (T + 1) & 1;
+          if (!wait_phase<kSpin>(&tfull[an], ((T + 1) >> 1) & 1, abort_flag, p.status, limit)) aborted = true;
+          tc_fence_after();
+          const uint32_t coln = lane_addr + an * N + g * RW * H;
+          tmem_ld32(coln, xa);
+          tmem_ld32(coln + 32, xb);
         }
 
         if (MODE == kModeLogits) {
@@ -1302,6 +1330,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
           }
         }
       }
+      tmem_ld_wait();  // no TMEM load of this warp stays in flight past its tile loop
       // (an aborted warp carries on to the next unit's group vote, which ends
       // the loop for every warp of the group together)
       if (MODE == kModeTopK) {
@@ -1532,6 +1561,7 @@ __global__ void fill_empty_kernel(int32_t* out_idx, float* out_vals, int64_t tot
 
 template <int R, bool PAGED, int H, int MODE>
 static cudaError_t launch_indexer(const IndexerParams& p, int grid, cudaStream_t st) {
+  static_assert(smem_layout<R, PAGED, H>().total + 1024 <= 227 * 1024, "shared memory per CTA");
   const size_t smem = static_cast<size_t>(smem_layout<R, PAGED, H>().total) + 1024;
   auto kern = indexer_kernel<R, PAGED, H, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
