@@ -883,6 +883,12 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
       for (int n = 0; ok; ++n) {
         const int qs = n & 3;
         if (!wait_phase<kSleep>(&uq_empty[qs], ((n >> 2) & 1) ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
+        // Claim only once a q slot is free, i.e. once the MMA is done with the
+        // unit before last: a CTA then holds at most one unit beyond the one
+        // in flight, so that at the end no CTA sits on work another could do.
+        // (An empty unit leaves its slot free; the next wait passes at once.)
+        const int qs2 = nq & 1;
+        if (!wait_phase<kProd>(&qempty[qs2], ((nq >> 1) & 1) ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
         int u = -1;
         if (p.repair_mode) {  // the groups the checks listed, one unit each (whole rows)
           const int idx = atomicAdd(p.status + kRepairSched, 1);
@@ -900,8 +906,6 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
         if (u < 0) break;
         const Unit U = get_unit<R, PAGED>(p, u);
         if (U.ntiles == 0) continue;
-        const int qs2 = nq & 1;
-        if (!wait_phase<kProd>(&qempty[qs2], ((nq >> 1) & 1) ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
         ++nq;
         mbar_arrive_expect_tx(&qfull[qs2], C::Q_BYTES);
         tma_load_2d(q_smem + qs2 * C::Q_BYTES, &p.tmap_q, &qfull[qs2], 0, U.row0 * H);
@@ -1426,7 +1430,7 @@ struct DenseSrc {
 
 constexpr int kMergeWarps = 8;
 constexpr int kMergeMaxChunks = kMergeWarps * 32;  // one chunk count per thread
-constexpr int kMergeStage = 24576;                 // pairs a row can gather in shared memory (192 KB)
+constexpr int kMergeStage = 12288;                 // pairs a row can gather in shared memory (96 KB: two CTAs per SM)
 
 // One CTA per row.  The chunk counts are scanned into offsets; when the
 // row's surviving pairs fit, they are gathered densely into shared memory and
