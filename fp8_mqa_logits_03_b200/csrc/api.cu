@@ -267,8 +267,12 @@ Plan plan_prefill(int64_t m, int64_t n, int topk, int sms, int H = kHeads) {
   return pl;
 }
 
-// One unit per (request, key chunk); chunks sized so that about four units
-// land on every SM (context lengths differ, so many chunks are short or empty).
+// One unit per (request, key chunk); chunks of the longest context sized so
+// that about kPagedUnitsPerSm units land on every SM (context lengths differ,
+// so many chunks are short or empty).  Small units even out the end of the
+// schedule; a unit's rows start from the thresholds their earlier chunks
+// raised, so later chunks pass few candidates.
+constexpr int kPagedUnitsPerSm = 8;
 Plan plan_paged(int64_t B, int R, int max_blocks, int topk, int sms, int H = kHeads) {
   Plan pl;
   pl.H = H;
@@ -277,8 +281,8 @@ Plan plan_paged(int64_t B, int R, int max_blocks, int topk, int sms, int H = kHe
   const int64_t axis = static_cast<int64_t>(max_blocks) * kPageSize;
   pl.chunk_keys = static_cast<int>(round_up(axis, kBlockKeys));
   pl.n_chunks = 1;
-  if (B < 4 * static_cast<int64_t>(sms)) {
-    const int64_t want = ceil_div(4 * static_cast<int64_t>(sms), B);
+  if (B < kPagedUnitsPerSm * static_cast<int64_t>(sms)) {
+    const int64_t want = ceil_div(kPagedUnitsPerSm * static_cast<int64_t>(sms), B);
     const int64_t ck = round_up(ceil_div(axis, want), kBlockKeys);
     pl.chunk_keys = static_cast<int>(ck);
     pl.n_chunks = static_cast<int>(ceil_div(axis, ck));

@@ -33,7 +33,8 @@ namespace {
 
 constexpr int kPrepThreads = 512;
 
-// Exclusive prefix sums of a[0..B) into off[0..B] by one CTA (B <= kMaxPrepBatch).
+// Exclusive prefix sums of a[0..B) into off[0..B] by one CTA (the caller bounds B
+// so that 2 (B + 1) int64 offsets fit in shared memory).
 __device__ void block_exclusive_scan(const int32_t* __restrict__ a, int B, int64_t* off, int64_t* warp_tot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int64_t carry = 0;
@@ -153,8 +154,6 @@ __global__ void transform_kernel(const int32_t* idx, int64_t rows, int topk,
 }
 
 }  // namespace
-
-constexpr int kMaxPrepBatch = 8192;
 
 cudaError_t launch_prepare_ragged(const int32_t* seq_len, const int32_t* q_len, const int32_t* req_idx, int B,
                                   const int32_t* table, int64_t table_rows, int64_t ld, int32_t* ks, int32_t* ke,

@@ -6,28 +6,29 @@
 //   out[i] = the top-k j of row i (larger L first, lower j on ties), padded with -1.
 //
 // Design (one persistent CTA per SM, warp-specialised):
-//   warp 0      TMA producer: the unit's q block [R rows x 32 heads x 128 B]
-//               once, then 128-key tiles [128 x 128 B] through a ring of
-//               shared-memory stages (paged keys: two 64-token pages a tile).
+//   warp 0      TMA producer: the unit's q block [R rows x H heads x 128 B]
+//               into one of two q slots, then 128-key tiles [128 x 128 B]
+//               through a ring of shared-memory stages (paged keys: two
+//               64-token pages a tile).
 //   warp 1      MMA issuer: tcgen05.mma kind::f8f6f4 with M = 128 keys,
-//               N = R*32 (row, head) columns, K = 128 as 4 x K32 steps, fp32
+//               N = R*H (row, head) columns, K = 128 as 4 x K32 steps, fp32
 //               accumulators in TMEM, double buffered (2 x N columns).
-//   warps 2..9  epilogue, two warpgroups of 4 (one warp per TMEM lane
-//               quadrant, so one thread per key); warpgroup g owns rows
-//               [g*R/2, (g+1)*R/2) of the unit.  Each thread reads its key's
-//               32 head dots per row from TMEM, applies ReLU, the head
-//               weights and the key scale, then either writes the logit
-//               (mqa_logits) or filters it against the row's running
-//               threshold into a per-row candidate buffer (fused top-k).
-//               A 512-bin histogram of each row's candidates (window opened
-//               on the row's first candidates) raises the threshold to the
-//               lower edge of the bin that holds the k-th candidate.
-//   warps 10..11 select group (fused top-k): takes a finished unit's row
+//   warps 2..3  select group (fused top-k): takes a finished unit's row
 //               state (double buffered, so it overlaps the next unit) and
 //               selects each row's exact top-k: keys above the boundary bin
 //               go straight out, the boundary bin is resolved in shared memory.
 //               Rows are claimed from a per-slot counter; once out of units,
-//               the first epilogue warpgroup claims the last units' rows too.
+//               the epilogue warps claim the last units' rows too.
+//   warps 4..   epilogue, warpgroups of 4 (one warp per TMEM lane quadrant,
+//               so one thread per key), each owning RW rows of the unit.  Each
+//               thread reads its key's head dots per row from TMEM, applies
+//               ReLU, the head weights and the key scale, then either writes
+//               the logit (mqa_logits) or filters it against the row's
+//               running threshold into its own segment of the row's
+//               candidate buffer (fused top-k).  At votes every few tiles a
+//               warp counts what it appended into the row's 512-bin
+//               histogram and raises the threshold to a lower bound on (or a
+//               checked estimate of) the row's k-th value.
 // A unit is R query rows (a row block, or one request's rows in the paged
 // form) times one chunk of keys, claimed from a device counter by the
 // producer and passed on through a shared-memory queue.  With one chunk per
@@ -269,69 +270,34 @@ __device__ __forceinline__ uint32_t bar_red_popc(int id, int nthreads, bool pred
   return r;
 }
 
-// 2 * sum_h w[h] * max(x[h], 0) over the 32 heads of one (key, row), as
-// sum_h (w[h] * x[h] + w[h] * |x[h]|): the identity 2 max(x, 0) = x + |x| keeps
-// the whole reduction on the FMA pipe (|x| is a free operand modifier) and off
-// the half-rate min/max pipe.  The linear half uses packed two-lane FMAs.
-// Each FMA rounds once; the extra rounding against the max form is a few
-// units in the last place of the running sum.  Callers scale by 0.5.
-__device__ __forceinline__ float relu_dot32_x2(const uint32_t (&x)[32], const float* wsm) {
-  const float4* w4 = reinterpret_cast<const float4*>(wsm);
-  uint64_t lin0 = 0, lin1 = 0;
-  float ab0 = 0.f, ab1 = 0.f, ab2 = 0.f, ab3 = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 wv = w4[i];
-    const float x0 = __uint_as_float(x[4 * i + 0]), x1 = __uint_as_float(x[4 * i + 1]);
-    const float x2 = __uint_as_float(x[4 * i + 2]), x3 = __uint_as_float(x[4 * i + 3]);
-    lin0 = fma_f32x2(pack_f32x2(wv.x, wv.y), pack_f32x2(x0, x1), lin0);
-    lin1 = fma_f32x2(pack_f32x2(wv.z, wv.w), pack_f32x2(x2, x3), lin1);
-    ab0 = fmaf(wv.x, fabsf(x0), ab0);
-    ab1 = fmaf(wv.y, fabsf(x1), ab1);
-    ab2 = fmaf(wv.z, fabsf(x2), ab2);
-    ab3 = fmaf(wv.w, fabsf(x3), ab3);
-  }
-  float l0, l1, l2, l3;
-  unpack_f32x2(lin0, l0, l1);
-  unpack_f32x2(lin1, l2, l3);
-  return ((l0 + ab0) + (l1 + ab1)) + ((l2 + ab2) + (l3 + ab3));
-}
-
-// relu_dot32_x2 for two rows at once, written so that the two rows' twelve
-// accumulator chains interleave (an FMA waits on its own chain only).
-__device__ __forceinline__ void relu_dot32_x2_pair(const uint32_t (&xa)[32], const uint32_t (&xb)[32],
-                                                   const float* wa, const float* wb, float& ra, float& rb) {
+// sum_h w[h] * max(x[h], 0) over the 32 heads of one (key, row), for two
+// rows at once.  The max runs on the ALU pipe and the weighted sum as packed
+// two-lane FMAs (fma.rn.f32x2), so each head costs one ALU issue and half an
+// FMA issue.  Two packed accumulators per row (heads 4i, 4i+1 and 4i+2,
+// 4i+3) give four independent FMA chains; a packed add and one add join a
+// row's four partial sums.  Each operation rounds once.
+__device__ __forceinline__ void relu_dot32_pair(const uint32_t (&xa)[32], const uint32_t (&xb)[32],
+                                                const float* wa, const float* wb, float& ra, float& rb) {
   const float4* wa4 = reinterpret_cast<const float4*>(wa);
   const float4* wb4 = reinterpret_cast<const float4*>(wb);
   uint64_t la0 = 0, la1 = 0, lb0 = 0, lb1 = 0;
-  float aa0 = 0.f, aa1 = 0.f, aa2 = 0.f, aa3 = 0.f, ab0 = 0.f, ab1 = 0.f, ab2 = 0.f, ab3 = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 va = wa4[i], vb = wb4[i];
-    const float a0 = __uint_as_float(xa[4 * i + 0]), a1 = __uint_as_float(xa[4 * i + 1]);
-    const float a2 = __uint_as_float(xa[4 * i + 2]), a3 = __uint_as_float(xa[4 * i + 3]);
-    const float b0 = __uint_as_float(xb[4 * i + 0]), b1 = __uint_as_float(xb[4 * i + 1]);
-    const float b2 = __uint_as_float(xb[4 * i + 2]), b3 = __uint_as_float(xb[4 * i + 3]);
+    const float a0 = fmaxf(__uint_as_float(xa[4 * i + 0]), 0.f), a1 = fmaxf(__uint_as_float(xa[4 * i + 1]), 0.f);
+    const float a2 = fmaxf(__uint_as_float(xa[4 * i + 2]), 0.f), a3 = fmaxf(__uint_as_float(xa[4 * i + 3]), 0.f);
+    const float b0 = fmaxf(__uint_as_float(xb[4 * i + 0]), 0.f), b1 = fmaxf(__uint_as_float(xb[4 * i + 1]), 0.f);
+    const float b2 = fmaxf(__uint_as_float(xb[4 * i + 2]), 0.f), b3 = fmaxf(__uint_as_float(xb[4 * i + 3]), 0.f);
     la0 = fma_f32x2(pack_f32x2(va.x, va.y), pack_f32x2(a0, a1), la0);
     lb0 = fma_f32x2(pack_f32x2(vb.x, vb.y), pack_f32x2(b0, b1), lb0);
     la1 = fma_f32x2(pack_f32x2(va.z, va.w), pack_f32x2(a2, a3), la1);
     lb1 = fma_f32x2(pack_f32x2(vb.z, vb.w), pack_f32x2(b2, b3), lb1);
-    aa0 = fmaf(va.x, fabsf(a0), aa0);
-    ab0 = fmaf(vb.x, fabsf(b0), ab0);
-    aa1 = fmaf(va.y, fabsf(a1), aa1);
-    ab1 = fmaf(vb.y, fabsf(b1), ab1);
-    aa2 = fmaf(va.z, fabsf(a2), aa2);
-    ab2 = fmaf(vb.z, fabsf(b2), ab2);
-    aa3 = fmaf(va.w, fabsf(a3), aa3);
-    ab3 = fmaf(vb.w, fabsf(b3), ab3);
   }
-  float a_l0, a_l1, a_l2, a_l3, b_l0, b_l1, b_l2, b_l3;
-  unpack_f32x2(la0, a_l0, a_l1);
-  unpack_f32x2(la1, a_l2, a_l3);
-  unpack_f32x2(lb0, b_l0, b_l1);
-  unpack_f32x2(lb1, b_l2, b_l3);
-  ra = ((a_l0 + aa0) + (a_l1 + aa1)) + ((a_l2 + aa2) + (a_l3 + aa3));
-  rb = ((b_l0 + ab0) + (b_l1 + ab1)) + ((b_l2 + ab2) + (b_l3 + ab3));
+  float p0, p1, q0, q1;
+  unpack_f32x2(add_f32x2(la0, la1), p0, p1);
+  unpack_f32x2(add_f32x2(lb0, lb1), q0, q1);
+  ra = p0 + p1;
+  rb = q0 + q1;
 }
 
 // (Only meaningful for key >= base; any other key maps to some bin in range.)
@@ -670,6 +636,42 @@ __device__ __forceinline__ int fold_segment(const uint2* seg, int from, int to, 
     }
   }
   return to;
+}
+
+// Count the candidates each of a warp's RW rows appended since the last
+// vote into the rows' histograms.  The common case (at most 128 new keys per
+// row) issues every row's loads before any count, so the read-back costs one
+// L2 round trip per vote; a row whose window is still closed, or that
+// appended more, goes through fold_segment.
+template <int RW>
+__device__ __forceinline__ void fold_rows(const uint2* seg0, int cap, int (&folded)[RW], const int (&cnt)[RW],
+                                          RowState* rs, uint32_t* hs, int lane) {
+  __syncwarp();  // the warp's own appends are visible to all its lanes
+  uint32_t kk[RW][4];
+#pragma unroll
+  for (int r = 0; r < RW; ++r) {
+    const uint2* seg = seg0 + static_cast<size_t>(r) * cap;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = folded[r] + i * 32 + lane;
+      kk[r][i] = e < cnt[r] ? seg[e].x : 0u;
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < RW; ++r) {
+    if (folded[r] >= cnt[r]) continue;
+    const Window w = window_of(ld_volatile_u64(&rs[r].win));
+    if (!w.open || cnt[r] - folded[r] > 4 * 32) {
+      folded[r] = fold_segment(seg0 + static_cast<size_t>(r) * cap, folded[r], cnt[r], rs + r, hs + r * kNB, lane);
+      continue;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = folded[r] + i * 32 + lane;
+      if (e < cnt[r] && kk[r][i] >= w.base) atomicAdd(&hs[r * kNB + hist_bin(kk[r][i], w.base, w.shift)], 1u);
+    }
+    folded[r] = cnt[r];
+  }
 }
 
 // A contiguous candidate list as a select source.
@@ -1104,7 +1106,10 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
         if (tid_wg < RW) {
           RowState& st = rs[tid_wg];
           st.wcnt[0] = st.wcnt[1] = st.wcnt[2] = st.wcnt[3] = 0;
-          st.theta = 0;
+          // with a split key axis a unit starts from the row's shared bound,
+          // which the row's other chunks may have raised already
+          const int rl = g * RW + tid_wg;
+          st.theta = p.n_chunks > 1 && rl < U.nrows ? ld_volatile_u32(p.row_theta + U.row0 + rl) : 0u;
           st.theta_spec = 0;
           st.win = 0ull;
         }
@@ -1138,10 +1143,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
       // ---- this warp's registers per row: candidates in its segment, how many of
       // them the row's histogram has counted, the key range, and the threshold
       // (reloaded from the row state at every vote)
-      // and the row's histogram window as this warp knows it (hbase = ~0 while
-      // closed: no key counts)
-      int cnt[RW], folded[RW], lo[RW], span[RW], hshift[RW];
-      uint32_t hbase[RW];
+      int cnt[RW], folded[RW], lo[RW], span[RW];
       float thf[RW];
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
@@ -1149,9 +1151,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
         folded[r] = 0;
         lo[r] = rs[r].lo;
         span[r] = rs[r].hi - rs[r].lo;
-        thf[r] = -INFINITY;
-        hbase[r] = 0xFFFFFFFFu;
-        hshift[r] = 0;
+        thf[r] = MODE == kModeTopK ? theta_float(rs[r].theta) : -INFINITY;
       }
       uint2* seg0 = MODE == kModeTopK ? cand_s + qd * wcap : nullptr;  // row r's segment: seg0 + r * cap
       uint32_t gseen = 0;  // split key axis: the row's shared bound as read at this warp's last vote
@@ -1185,7 +1185,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
       }
       for (int t = 0; t < U.ntiles; ++t, ++T) {
         const int j = key0 + t * kBlockKeys;
-        const float sj = 0.5f * s_next;  // relu_dot32_x2 returns twice the head sum
+        const float sj = s_next;
         s_next = scale_of(j + kBlockKeys);  // (0 past the end)
         const uint32_t a = T & 1;
         // The last wait leaves the whole accumulator in registers: release it
@@ -1206,17 +1206,17 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
             tc_fence_before();
             __syncwarp();
             mbar_arrive_if(lane == 0, &tempty[a]);
-            relu_dot32_x2_pair(xa, xb, ws_g, ws_g + 32, Lc[0], Lc[1]);
+            relu_dot32_pair(xa, xb, ws_g, ws_g + 32, Lc[0], Lc[1]);
           } else {
             uint32_t xc[32], xd[32];
             tmem_ld32(col0 + 64, xc);
             tmem_ld32(col0 + 96, xd);
-            relu_dot32_x2_pair(xa, xb, ws_g, ws_g + 32, Lc[0], Lc[1]);
+            relu_dot32_pair(xa, xb, ws_g, ws_g + 32, Lc[0], Lc[1]);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             mbar_arrive_if(lane == 0, &tempty[a]);
-            relu_dot32_x2_pair(xc, xd, ws_g + 64, ws_g + 96, Lc[2], Lc[NC - 1]);
+            relu_dot32_pair(xc, xd, ws_g + 64, ws_g + 96, Lc[2], Lc[NC - 1]);
           }
         }
         float L[RW];
@@ -1245,10 +1245,10 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
           }
           if (aborted) break;
         } else {
-          // ---- filter against the row's threshold; append to this warp's segment
-          // and count the key into the row's histogram (once its window is open).
-          // Stage by stage over the rows, so that the rows' chains interleave
-          // ahead of the stores (which keep their order).
+          // ---- filter against the row's threshold and append to this warp's
+          // segment (the row's histogram counts them at the next vote).  Stage by
+          // stage over the rows, so that the rows' chains interleave ahead of
+          // the stores (which keep their order).
           bool ps[RW];
           uint32_t key[RW], msk[RW];
 #pragma unroll
@@ -1259,19 +1259,16 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
 #pragma unroll
           for (int r = 0; r < RW; ++r) msk[r] = __ballot_sync(0xFFFFFFFFu, ps[r]);
           int pos[RW];
-          uint32_t* hp[RW];
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
             pos[r] = cnt[r] + __popc(msk[r] & lt);
             cnt[r] += __popc(msk[r]);
-            hp[r] = hs + r * kNB + hist_bin(key[r], hbase[r], hshift[r]);
           }
 #pragma unroll
           for (int r = 0; r < RW; ++r)
             st_global_v2_if(ps[r] && pos[r] < wcap, seg0 + static_cast<size_t>(r) * cap + pos[r], key[r],
                             static_cast<uint32_t>(j));
-#pragma unroll
-          for (int r = 0; r < RW; ++r) red_shared_add_if(ps[r] && key[r] >= hbase[r], hp[r], 1u);
+
           // ---- vote: count, make room, reload the thresholds (this warp alone)
           if (t == next_vote || t + 1 == U.ntiles) {
             const int vnext = vote_interval(t + 1);
@@ -1286,18 +1283,9 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
             for (int r = 0; r < RW; ++r) {
               if (cnt[r] > wcap && lane == 0) atomicOr(p.status, kStatusCandOverflow);
               cnt[r] = min(cnt[r], wcap);
-              if (hbase[r] == 0xFFFFFFFFu && cnt[r] > 0) {
-                // once per row: open the window (or take the one another warp
-                // opened) and count what was appended before it
-                folded[r] = fold_segment(seg0 + static_cast<size_t>(r) * cap, folded[r], cnt[r], rs + r,
-                                         hs + r * kNB, lane);
-                const Window w = window_of(ld_volatile_u64(&rs[r].win));
-                hbase[r] = w.base;
-                hshift[r] = w.shift;
-              }
-              folded[r] = cnt[r];  // the hot loop counts from here on
               full |= cnt[r] + room > wcap;
             }
+            fold_rows<RW>(seg0, cap, folded, cnt, rs, hs, lane);
             while (full) {  // rare: one row at a time, through a single copy of the compaction
               int cr = -1, cc = 0;
 #pragma unroll
@@ -1315,9 +1303,11 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
                 if (r == cr) cnt[r] = folded[r] = nc;
             }
             if (qd < RW && g * RW + qd < U.nrows) {
-              // this warp keeps the threshold of the group's row qd; an estimate
-              // counts the row's keys in tiles [0, t + 1] as seen (the other
-              // warps may be a tile ahead), which only lowers it
+              // this warp keeps the threshold of the group's row qd.  An estimate
+              // takes the row's keys in tiles [0, t + 1] as seen.  Another warp
+              // may already have counted tile t + 2 (this warp has released
+              // tile t's accumulator), which makes the estimate a little
+              // bolder; like any estimate it is checked against the result.
               const RowState* me = rs + qd;
               int target = k;
               if (p.speculate) {

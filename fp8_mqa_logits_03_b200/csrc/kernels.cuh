@@ -20,7 +20,7 @@ constexpr int kStatusBytes = 256;  // device status block at the head of every w
 // growing with the tiles already streamed (clamp(t / 4, min, max)), since the
 // threshold's relative movement per tile falls like 1 / t.
 constexpr int kMinVoteTiles = 4;
-constexpr int kMaxVoteTiles = 16;
+constexpr int kMaxVoteTiles = 32;
 __host__ __device__ constexpr int vote_interval(int t) {
   return t / 4 < kMinVoteTiles ? kMinVoteTiles : (t / 4 > kMaxVoteTiles ? kMaxVoteTiles : t / 4);
 }

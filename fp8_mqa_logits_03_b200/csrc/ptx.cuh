@@ -85,6 +85,13 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
   return d;
 }
 
+// (a.lo + b.lo, a.hi + b.hi), each rounded once to nearest.
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -109,20 +116,14 @@ __device__ __forceinline__ void l2_prefetch_bulk(const void* src, uint32_t bytes
                : "memory");
 }
 
-// Predicated stores and reductions: one instruction under a predicate, so
-// that a per-lane condition costs no branch.  No memory clobber: callers
-// order them against later readers with a barrier.
+// Predicated store: one instruction under a predicate, so that a per-lane
+// condition costs no branch.  No memory clobber: callers order it against
+// later readers with a barrier.
 __device__ __forceinline__ void st_global_v2_if(bool pred, void* p, uint32_t a, uint32_t b) {
   asm volatile(
       "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t@q st.global.v2.u32 [%1], {%2, %3};\n\t}" ::"r"(
           static_cast<uint32_t>(pred)),
       "l"(reinterpret_cast<uint64_t>(p)), "r"(a), "r"(b));
-}
-__device__ __forceinline__ void red_shared_add_if(bool pred, uint32_t* p, uint32_t v) {
-  asm volatile(
-      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t@q red.shared.add.u32 [%1], %2;\n\t}" ::"r"(
-          static_cast<uint32_t>(pred)),
-      "r"(smem_u32(p)), "r"(v));
 }
 
 // ---------------------------------------------------------------- named barriers
