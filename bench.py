@@ -393,6 +393,11 @@ def time_device(call, steps: int, warmup: int, flush, stream):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     torch.cuda.synchronize()
+    # an untimed spin of about a millisecond first, so that the host has the
+    # next steps queued before the GPU reaches them: a host-side delay then
+    # cannot leave the GPU idle inside a timed step
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(2_000_000)
     for i in range(steps):
         flush.zero_()
         starts[i].record(stream)
