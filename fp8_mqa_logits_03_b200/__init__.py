@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
             L.fp8idx_paged_mqa_logits_topk_workspace.restype = sz
             L.fp8idx_paged_mqa_logits_topk.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, i64,
                                                        i32, i32, i32, i32, vp, vp, vp, sz, vp]
+            L.fp8idx_paged_mqa_logits_topk_slots.argtypes = L.fp8idx_paged_mqa_logits_topk.argtypes
             L.fp8idx_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
             L.fp8idx_read_device_stats.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), i32, vp]
             L.fp8idx_read_device_stats.restype = ctypes.c_int
@@ -79,7 +80,8 @@ def lib() -> ctypes.CDLL:
                                                 vp]
             L.fp8idx_topk_transform.argtypes = [vp, i64, i32, vp, vp, i32, vp, i64, i64, i32, vp, vp]
             for name in ("fp8idx_mqa_logits", "fp8idx_topk_rows", "fp8idx_mqa_logits_topk",
-                         "fp8idx_paged_mqa_logits_topk", "fp8idx_read_device_status",
+                         "fp8idx_paged_mqa_logits_topk", "fp8idx_paged_mqa_logits_topk_slots",
+                         "fp8idx_read_device_status",
                          "fp8idx_act_quant_store", "fp8idx_prepare_ragged", "fp8idx_topk_transform"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
@@ -233,8 +235,11 @@ def mqa_logits_topk(q, k, s, w, ks, ke, topk: int = MAX_TOPK, out=None, out_vals
 
 def paged_mqa_logits_topk(q, k_pages, s_pages, w, block_table, seq_lens, R: int,
                           topk: int = MAX_TOPK, out=None, out_vals=None, workspace=None,
-                          return_values: bool = False, stream=None):
-    """Paged decode/verify: R rows per request, keys through a 64-token block table."""
+                          return_values: bool = False, stream=None, slots: bool = False):
+    """Paged decode/verify: R rows per request, keys through a 64-token block table.
+
+    slots=True returns physical KV slots (block_table[b, j // 64] * 64 + j % 64)
+    instead of logical positions j, mapped where the indices are written."""
     q = _bytes(q, "q")
     k_pages = _bytes(k_pages, "k_pages")
     s_pages = _dev(s_pages, "s_pages", torch.float32)
@@ -254,11 +259,10 @@ def paged_mqa_logits_topk(q, k_pages, s_pages, w, block_table, seq_lens, R: int,
     need = paged_workspace_size(B, R, max_blocks, topk, q.shape[1])
     if workspace is None:
         workspace = alloc_workspace(need, q.device)
-    _check(lib().fp8idx_paged_mqa_logits_topk(_ptr(q), _ptr(k_pages), _ptr(s_pages), _ptr(w),
-                                              _ptr(block_table), _ptr(seq_lens), B, R, max_blocks,
-                                              num_pages, page_size, q.shape[1], q.shape[2], topk,
-                                              _ptr(out), _ptr(out_vals), _ptr(workspace),
-                                              workspace.numel(), _stream(stream)))
+    fn = lib().fp8idx_paged_mqa_logits_topk_slots if slots else lib().fp8idx_paged_mqa_logits_topk
+    _check(fn(_ptr(q), _ptr(k_pages), _ptr(s_pages), _ptr(w), _ptr(block_table), _ptr(seq_lens), B, R,
+              max_blocks, num_pages, page_size, q.shape[1], q.shape[2], topk, _ptr(out), _ptr(out_vals),
+              _ptr(workspace), workspace.numel(), _stream(stream)))
     return (out, out_vals) if return_values else out
 
 

@@ -223,7 +223,8 @@ int run_fused_topk(const Plan& pl, IndexerParams& p, uint8_t* wsb, bool paged, i
   if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
   if (pl.n_chunks > 1) {
     MergeParams mp{p.part, p.part_cnt, static_cast<int>(rows), pl.rows_per_unit, pl.R, pl.n_chunks, topk,
-                   p.out_idx, p.out_vals, p.row_spec, p.status, p.repair_flag, p.repair_list};
+                   p.out_idx, p.out_vals, p.row_spec, p.status, p.repair_flag, p.repair_list,
+                   p.out_slots ? p.block_table : nullptr, p.max_blocks, p.num_pages};
     e = launch_merge(mp, st);
     if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }
@@ -505,12 +506,11 @@ size_t fp8idx_paged_mqa_logits_topk_workspace(int64_t B, int R, int max_blocks, 
   return plan_paged(std::max<int64_t>(B, 1), R, max_blocks, topk, sms, H).total;
 }
 
-int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const float* s_pages,
-                                 const float* w, const int32_t* block_table,
-                                 const int32_t* seq_lens, int64_t B, int R, int max_blocks,
-                                 int64_t num_pages, int page_size, int H, int D, int topk,
-                                 int32_t* out_idx, float* out_vals, void* ws, size_t ws_bytes,
-                                 void* stream) {
+// The paged call; out_slots: write physical KV slots instead of positions.
+static int paged_topk(const uint8_t* q, const uint8_t* k_pages, const float* s_pages, const float* w,
+               const int32_t* block_table, const int32_t* seq_lens, int64_t B, int R, int max_blocks,
+               int64_t num_pages, int page_size, int H, int D, int topk, int32_t* out_idx, float* out_vals,
+               void* ws, size_t ws_bytes, void* stream, bool out_slots) {
   FP8IDX_TRY(check_shape(H, D));
   FP8IDX_TRY(check_topk(topk));
   if (page_size != kPageSize) return fail(FP8IDX_EUNSUPPORTED, "page_size must be 64 (got %d)", page_size);
@@ -558,7 +558,28 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
   p.topk = topk;
   p.out_idx = out_idx;
   p.out_vals = out_vals;
+  p.out_slots = out_slots ? 1 : 0;
   return run_fused_topk(pl, p, wsb, true, B * R, st);
+}
+
+int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const float* s_pages,
+                                 const float* w, const int32_t* block_table,
+                                 const int32_t* seq_lens, int64_t B, int R, int max_blocks,
+                                 int64_t num_pages, int page_size, int H, int D, int topk,
+                                 int32_t* out_idx, float* out_vals, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  return paged_topk(q, k_pages, s_pages, w, block_table, seq_lens, B, R, max_blocks, num_pages, page_size, H, D,
+                    topk, out_idx, out_vals, ws, ws_bytes, stream, false);
+}
+
+int fp8idx_paged_mqa_logits_topk_slots(const uint8_t* q, const uint8_t* k_pages, const float* s_pages,
+                                       const float* w, const int32_t* block_table,
+                                       const int32_t* seq_lens, int64_t B, int R, int max_blocks,
+                                       int64_t num_pages, int page_size, int H, int D, int topk,
+                                       int32_t* out_slots, float* out_vals, void* ws, size_t ws_bytes,
+                                       void* stream) {
+  return paged_topk(q, k_pages, s_pages, w, block_table, seq_lens, B, R, max_blocks, num_pages, page_size, H, D,
+                    topk, out_slots, out_vals, ws, ws_bytes, stream, true);
 }
 
 // Allocation-free form of fp8idx_mqa_logits_topk for callers that cannot

@@ -552,9 +552,13 @@ __device__ void write_row_topk(const IndexerParams& p, const SlotMeta& meta, int
     int32_t* orow = p.out_idx + static_cast<int64_t>(row) * k;
     float* vrow = p.out_vals ? p.out_vals + static_cast<int64_t>(row) * k : nullptr;
     uint32_t vmin = 0xFFFFFFFFu;  // the smallest order key written (this thread's share)
+    const int req = row / p.rows_per_unit;  // paged: the row's request
     const int nout = final_select_row<FAST>(rowbuf, wcap, st, h, k, g, up_all, at_all, xchg, p.status,
                                             [&](int pos, uint32_t key, uint32_t j) {
-                                              orow[pos] = static_cast<int32_t>(j);
+                                              orow[pos] = p.out_slots ? slot_of(p.block_table, p.max_blocks,
+                                                                                p.num_pages, req,
+                                                                                static_cast<int32_t>(j))
+                                                                      : static_cast<int32_t>(j);
                                               if (vrow) vrow[pos] = key_to_float(key);
                                               vmin = min(vmin, key);
                                             });
@@ -1466,7 +1470,8 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
   float* vrow = p.out_vals ? p.out_vals + static_cast<int64_t>(row) * p.topk : nullptr;
   uint32_t vmin = 0xFFFFFFFFu;  // the smallest order key written (this thread's share)
   auto emit = [&](int pos, uint64_t K) {
-    orow[pos] = static_cast<int32_t>(composite_index(K));
+    const int32_t j = static_cast<int32_t>(composite_index(K));
+    orow[pos] = p.block_table ? slot_of(p.block_table, p.max_blocks, p.num_pages, unit_row, j) : j;
     if (vrow) vrow[pos] = key_to_float(composite_value(K));
     vmin = min(vmin, composite_value(K));
   };

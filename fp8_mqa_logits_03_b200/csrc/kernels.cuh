@@ -85,6 +85,7 @@ struct IndexerParams {
   int* repair_flag;     // [row blocks / requests]: listed for recomputation (zeroed per call)
   int* repair_list;     // [row blocks / requests]
   int repair_mode;      // this launch recomputes the listed groups, whole rows, exact thresholds
+  int out_slots;        // paged: write physical KV slots (block_table[b][j / 64] * 64 + j % 64), not positions j
 };
 
 struct MergeParams {
@@ -101,7 +102,19 @@ struct MergeParams {
   int* status;               // the call's status block (repair count and stats)
   int* repair_flag;
   int* repair_list;
+  const int32_t* block_table;  // non-null: write physical KV slots through this [requests, max_blocks] table
+  int max_blocks;
+  int num_pages;
 };
+
+// Physical KV slot of logical key position j of request b through a block
+// table of 64-token pages: -1 for j < 0 or a page entry outside the pool.
+__device__ __forceinline__ int32_t slot_of(const int32_t* block_table, int max_blocks, int num_pages, int b,
+                                           int32_t j) {
+  if (j < 0) return -1;
+  const int32_t pg = __ldg(block_table + static_cast<int64_t>(b) * max_blocks + j / kPageSize);
+  return pg >= 0 && pg < num_pages ? pg * kPageSize + j % kPageSize : -1;
+}
 
 struct TopkRowsParams {
   const float* logits;

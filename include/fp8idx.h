@@ -138,6 +138,24 @@ int fp8idx_paged_mqa_logits_topk(const uint8_t* q, const uint8_t* k_pages, const
                                  void* stream);
 
 /*
+ * fp8idx_paged_mqa_logits_topk with the top-k transform applied where the
+ * indices are written: each selected position j of request b comes out as
+ * its physical KV slot block_table[b, j / 64] * 64 + j % 64, the slot the
+ * sparse attention reads (the paged form of `fast_topk_transform_fused`'s
+ * page-table mapping on the "bench_mqa_logits_chunking.py" page).  -1
+ * padding stays -1; a selected key on a page entry outside [0, num_pages)
+ * (which also sets the BAD_PAGE status bit) comes out as -1.  Same
+ * arguments, workspace size, ownership and errors as
+ * fp8idx_paged_mqa_logits_topk; the values in out_vals are unchanged.
+ */
+int fp8idx_paged_mqa_logits_topk_slots(const uint8_t* q, const uint8_t* k_pages, const float* s_pages,
+                                       const float* w, const int32_t* block_table,
+                                       const int32_t* seq_lens, int64_t B, int R, int max_blocks,
+                                       int64_t num_pages, int page_size, int H, int D, int topk,
+                                       int32_t* out_slots, float* out_vals, void* ws, size_t ws_bytes,
+                                       void* stream);
+
+/*
  * Allocation-free variant of fp8idx_mqa_logits_topk (the pages have no
  * counterpart: it exists for callers that cannot allocate device memory at
  * call time, such as code inside a framework-owned CUDA graph or a runtime

@@ -5,8 +5,10 @@ import pytest
 import torch
 
 from oracle import index_prep as ip
+from oracle import paged_logits_rows
 import fp8_mqa_logits_03_b200 as fx
 from fp8_mqa_logits_03_b200 import workloads
+from _parity import check_topk_row, paged_range
 
 pytestmark = pytest.mark.gpu
 
@@ -99,15 +101,53 @@ def test_transform_ragged_matches_oracle():
     assert np.array_equal(t_idx.cpu().numpy(), want)
 
 
-def test_transform_of_the_paged_topk_matches_oracle():
-    """The paged indexer's logical positions through its block table (64-token
-    pages): the kernel's own output, transformed on the GPU and by the oracle."""
+def test_transform_through_the_block_table_matches_oracle():
+    """Seeded top-k positions of paged rows (R rows per request, -1 padding)
+    through the paged form's block table of 64-token pages: GPU against oracle."""
     lengths = [5000, 300, 4200, 64, 2049]
     R, k = 4, 512
     d = workloads.make_paged(len(lengths), R, 1, 5000, seed=23, lengths=lengths)
-    t = {x: d[x].cuda() for x in ("q", "k_pages", "s_pages", "w", "block_table", "seq_lens")}
-    idx = fx.paged_mqa_logits_topk(**t, R=R, topk=k)
-    slots = fx.topk_transform(idx, t["block_table"], 64, rows_per_table_row=R)
-    want = ip.topk_transform(idx.cpu().numpy(), d["block_table"].numpy(), 64, rows_per_table_row=R)
+    g = np.random.default_rng(29)
+    idx = np.full((len(lengths) * R, k), -1, dtype=np.int32)
+    for row in range(idx.shape[0]):
+        L = lengths[row // R]
+        n = min(k, L)
+        idx[row, :n] = g.choice(L, size=n, replace=False)
+    want = ip.topk_transform(idx, d["block_table"].numpy(), 64, rows_per_table_row=R)
+    slots = fx.topk_transform(torch.from_numpy(idx).cuda(), d["block_table"].cuda(), 64, rows_per_table_row=R)
     assert np.array_equal(slots.cpu().numpy(), want)
-    assert np.all((slots.cpu().numpy() >= 0) == (idx.cpu().numpy() >= 0))
+    assert np.all((want >= 0) == (idx >= 0))
+
+
+@pytest.mark.parametrize("lengths,R,k", [
+    ([5000, 300, 4200, 64, 2049, 1, 129], 4, 2048),   # direct and short rows
+    ([9000, 7000, 130, 6000], 8, 512),                # MTP-8, top-512
+    ([3000] * 40, 1, 2048),                            # decode, many requests
+    ([200 + (i % 7) * 37 for i in range(1200)], 1, 64),  # enough requests for whole-row units (no merge)
+])
+def test_paged_topk_slots_match_oracle(lengths, R, k):
+    """The paged top-k written as physical KV slots (the transform applied
+    where the indices are emitted, in the fused kernel or the merge): each
+    slot maps back through the block table to a logical position that passes
+    the oracle's top-k check, and equals the oracle's transform of it."""
+    d = workloads.make_paged(len(lengths), R, 1, max(lengths), seed=31 + R, lengths=lengths)
+    t = {x: d[x].cuda() for x in ("q", "k_pages", "s_pages", "w", "block_table", "seq_lens")}
+    ws = fx.alloc_workspace(fx.paged_workspace_size(len(lengths), R, d["max_blocks"], k))
+    slots, vals = fx.paged_mqa_logits_topk(**t, R=R, topk=k, return_values=True, workspace=ws, slots=True)
+    assert fx.read_device_status(ws) == 0
+    slots, vals = slots.cpu().numpy(), vals.cpu().numpy()
+    bt = d["block_table"].numpy()
+    rows = np.arange(len(lengths) * R)
+    ref = paged_logits_rows(d["q"].numpy(), d["k_pages"].numpy(), d["s_pages"].numpy(), d["w"].numpy(), bt,
+                            d["seq_lens"].numpy(), R, rows=rows)
+    for row in rows:
+        b = row // R
+        L = int(lengths[b])
+        page_to_block = {int(pg): blk for blk, pg in enumerate(bt[b, :(L + 63) // 64])}
+        s = slots[row]
+        pos = np.array([-1 if x < 0 else page_to_block[int(x) // 64] * 64 + int(x) % 64 for x in s],
+                       dtype=np.int64)
+        lo, hi = paged_range(L, R, row % R)
+        check_topk_row(pos, ref[row], lo, hi, k, vals[row], f"row {row}")
+        want = ip.topk_transform(pos[None, :].astype(np.int32), bt[b:b + 1], 64)
+        assert np.array_equal(want[0], s), f"row {row}: slot differs from the oracle transform"
