@@ -524,8 +524,8 @@ static int paged_topk(const uint8_t* q, const uint8_t* k_pages, const float* s_p
   if (!q || !w || !block_table || !seq_lens || !out_idx)
     return fail(FP8IDX_EINVAL, "null q, w, block_table, seq_lens or out_idx");
   if (num_pages > 0 && (!k_pages || !s_pages)) return fail(FP8IDX_EINVAL, "null k_pages or s_pages");
-  if (!aligned(q, 16) || !aligned(k_pages, 16))
-    return fail(FP8IDX_EINVAL, "q and k_pages must be 16-byte aligned");
+  if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(s_pages, 16))
+    return fail(FP8IDX_EINVAL, "q, k_pages and s_pages must be 16-byte aligned");
   if (!aligned(s_pages, 4) || !aligned(w, 4) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
       !aligned(out_idx, 4) || !aligned(out_vals, 4))
     return fail(FP8IDX_EINVAL, "pointers must be 4-byte aligned");

@@ -44,6 +44,9 @@
 
 namespace fp8idx {
 
+// Key scales of a page that is not in the pool: zero (never written).
+__device__ __align__(128) float g_zero_scales[kPageSize];
+
 // Warp roles: warpgroup 0 holds the TMA producer (warp 0), the MMA issuer
 // (warp 1) and the select group (warps 2-3); then EWG epilogue warpgroups of
 // four warps, one per TMEM lane quadrant (warp % 4), each warpgroup owning RW
@@ -58,12 +61,17 @@ struct Cfg {
   static constexpr int EPI_WARPS = 4 * EWG;
   static constexpr int THREADS = 32 * (4 + EPI_WARPS);
   // key-tile ring depth: what shared memory leaves next to two q blocks
-  static constexpr int STAGES = R == 8 ? 4 : (H == 64 ? 5 : (PAGED ? 7 : 5));
+  static constexpr int STAGES = R == 8 ? 4 : (H == 64 ? 5 : (PAGED ? 6 : 5));
+  // paged: a ring of the tiles' key scales (two 64-token pages each), filled
+  // by the producer with bulk copies beside the key tiles; more entries than
+  // the producer can run ahead of the epilogue (STAGES + 2 tiles)
+  static constexpr int SRING = PAGED ? (STAGES + 3 <= 8 ? 8 : 16) : 0;
   static constexpr int Q_BYTES = N * kDim;
   static constexpr int TILE_BYTES = kBlockKeys * kDim;
   static constexpr int TMEM_COLS = 2 * N <= 256 ? 256 : 512;  // double-buffered accumulators
   static constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockKeys, N);
   static_assert(N <= 256 && N % 16 == 0, "MMA N out of range");
+  static_assert(!PAGED || SRING >= STAGES + 3, "scale ring shorter than the producer's lead");
   static_assert(R % RW == 0 && EPI_WARPS <= kMaxEpiWarps, "epilogue layout");
   static_assert(H % 32 == 0 && (NC == 2 || NC == 4), "32-column chunks per epilogue warp");
 };
@@ -120,7 +128,7 @@ struct SlotMeta {
 };
 
 struct SmemLayout {
-  int q, stage, bar, misc, w, rows, meta, hist, esel, ssel, up, at, total;
+  int q, stage, bar, misc, w, rows, meta, hist, esel, ssel, up, at, sring, total;
 };
 
 template <int R, bool PAGED, int H>
@@ -130,7 +138,7 @@ __host__ __device__ constexpr SmemLayout smem_layout() {
   L.q = 0;  // two q blocks: the next unit's loads while this unit's MMAs run
   L.stage = 2 * C::Q_BYTES;
   L.bar = L.stage + C::STAGES * C::TILE_BYTES;
-  L.misc = L.bar + 8 * (2 * C::STAGES + 22);
+  L.misc = L.bar + 8 * (2 * C::STAGES + 38);
   L.w = L.misc + 64;
   L.rows = L.w + R * H * 4;
   L.meta = L.rows + 2 * R * static_cast<int>(sizeof(RowState));
@@ -139,7 +147,8 @@ __host__ __device__ constexpr SmemLayout smem_layout() {
   L.ssel = L.esel + C::EPI_WARPS * kSelWords * 4;
   L.up = L.ssel + 320 * 4;
   L.at = L.up + kSelWarps * kUpCap * 8;
-  L.total = L.at + kSelWarps * kAtCap * 8;
+  L.sring = L.at + kSelWarps * kAtCap * 8;
+  L.total = L.sring + C::SRING * kBlockKeys * 4;
   return L;
 }
 
@@ -789,6 +798,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
   constexpr int N = C::N;
   constexpr int RW = C::RW;
   constexpr int S = C::STAGES;
+  constexpr uint32_t SR = C::SRING > 0 ? C::SRING : 1;  // scale ring entries (paged)
   static_assert(4 * (kUpCap + kAtCap) * 8 <= SL.stage + S * C::TILE_BYTES,
                 "end-of-kernel select staging must fit in the q and key-tile buffers");
 
@@ -810,6 +820,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
   uint64_t* slot_empty = bars + 2 * S + 11;
   uint64_t* uq_full = bars + 2 * S + 13;   // unit queue, 4 entries
   uint64_t* uq_empty = bars + 2 * S + 17;
+  uint64_t* sfull = bars + 2 * S + 21;     // paged: the scale ring (SRING entries)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SL.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL.misc + 4);
   volatile int* uq = reinterpret_cast<volatile int*>(smem + SL.misc + 16);  // unit queue
@@ -822,6 +833,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
   uint32_t* ssel_smem = reinterpret_cast<uint32_t*>(smem + SL.ssel);
   uint2* up_smem = reinterpret_cast<uint2*>(smem + SL.up);
   uint2* at_smem = reinterpret_cast<uint2*>(smem + SL.at);
+  float* sring = reinterpret_cast<float*>(smem + SL.sring);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -848,6 +860,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
       mbar_init(&qfull[x], 1);
       mbar_init(&qempty[x], 1);
     }
+    for (int x = 0; x < C::SRING; ++x) mbar_init(&sfull[x], 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -878,6 +891,8 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
         issued_phase[s] = 0;
       }
       bool ok = true;
+      uint32_t Tp = 0;                      // the CTA's tiles issued so far
+      uint32_t s_issued = 0, s_phase = 0;   // scale ring entries with a copy issued, and its phase
       // Dynamic schedule: units are claimed from a counter in the status block
       // and announced to the MMA and epilogue warps through a four-entry
       // queue; -1 ends the stream.  Whole-row units go last row block first
@@ -920,6 +935,12 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
           if (!wait_phase<kProd>(&empty[stage], phase ^ 1, abort_flag, p.status, limit)) { ok = false; break; }
           const int j0 = U.jbeg + t * kBlockKeys;
           uint8_t* dst = stage_smem + stage * C::TILE_BYTES;
+          // paged: the tile's two pages through the block table
+          const bool has1 = PAGED && j0 + kPageSize < U.len;
+          const int32_t pg0 = PAGED ? __ldg(bt + j0 / kPageSize) : -1;
+          const int32_t pg1 = has1 ? __ldg(bt + j0 / kPageSize + 1) : -1;
+          const bool v0 = pg0 >= 0 && pg0 < p.num_pages;
+          const bool v1 = has1 && pg1 >= 0 && pg1 < p.num_pages;
           if (p.debug_withhold_first_tile && n == 0 && t == 0) {
             // tests only: this stage never fills, so the MMA's bounded wait on
             // it runs out and the kernel takes its timeout path
@@ -927,17 +948,23 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
             mbar_arrive_expect_tx(&full[stage], C::TILE_BYTES);
             tma_load_2d(dst, &p.tmap_k, &full[stage], 0, j0);
           } else {
-            const int lp = j0 / kPageSize;
-            const bool has1 = j0 + kPageSize < U.len;
-            const int32_t pg0 = __ldg(bt + lp);
-            const int32_t pg1 = has1 ? __ldg(bt + lp + 1) : -1;
-            const bool v0 = pg0 >= 0 && pg0 < p.num_pages;
-            const bool v1 = has1 && pg1 >= 0 && pg1 < p.num_pages;
             if (!v0 || (has1 && !v1)) atomicOr(p.status, kStatusBadPage);
             mbar_arrive_expect_tx(&full[stage], (v0 ? 8192u : 0u) + (v1 ? 8192u : 0u));
             if (v0) tma_load_2d(dst, &p.tmap_k, &full[stage], 0, pg0 * kPageSize);
             if (v1) tma_load_2d(dst + 8192, &p.tmap_k, &full[stage], 0, pg1 * kPageSize);
           }
+          if (PAGED) {  // the tile's key scales into the ring (a page outside the pool: zeros)
+            const int e = static_cast<int>(Tp % SR);
+            float* sd = sring + e * kBlockKeys;
+            mbar_arrive_expect_tx(&sfull[e], has1 ? 512u : 256u);
+            bulk_load(sd, v0 ? p.s + static_cast<int64_t>(pg0) * kPageSize : g_zero_scales, 256u, &sfull[e]);
+            if (has1)
+              bulk_load(sd + kPageSize, v1 ? p.s + static_cast<int64_t>(pg1) * kPageSize : g_zero_scales, 256u,
+                        &sfull[e]);
+            s_issued |= 1u << e;
+            s_phase = (s_phase & ~(1u << e)) | (((Tp / SR) & 1u) << e);
+          }
+          ++Tp;
           issued[stage] = !(p.debug_withhold_first_tile && n == 0 && t == 0);
           issued_phase[stage] = phase;
           if (++stage == S) {
@@ -946,12 +973,20 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
           }
         }
       }
-      // Never leave a copy in flight: wait for every stage's last issued load.
+      // Never leave a copy in flight: wait for every stage's last issued load
+      // and every scale ring entry's last copy.
 #pragma unroll 1
       for (int s = 0; s < S; ++s) {
         if (!issued[s]) continue;
         const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(&full[s], issued_phase[s]) && global_timer_ns() - t0 < 200000000ull) {
+        }
+      }
+#pragma unroll 1
+      for (int e = 0; e < C::SRING; ++e) {
+        if (!((s_issued >> e) & 1u)) continue;
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(&sfull[e], (s_phase >> e) & 1u) && global_timer_ns() - t0 < 200000000ull) {
         }
       }
     }
@@ -1162,14 +1197,10 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
 
       // ---- stream the unit's key tiles
       const int key0 = U.jbeg + qd * 32 + lane;
-      auto scale_of = [&](int j) -> float {
-        if (!PAGED) return j < p.n ? __ldg(p.s + j) : 0.f;
-        if (j >= U.len) return 0.f;
-        const int32_t pg = __ldg(p.block_table + static_cast<int64_t>(U.req) * p.max_blocks + j / kPageSize);
-        if (pg < 0 || pg >= p.num_pages) return 0.f;
-        return __ldg(p.s + static_cast<int64_t>(pg) * kPageSize + (j % kPageSize));
-      };
-      float s_next = U.ntiles ? scale_of(key0) : 0.f;
+      // key scales: read a tile ahead from global memory; paged, from the
+      // producer's scale ring (the tile's pages are scattered over the pool)
+      auto scale_of = [&](int j) -> float { return j < p.n ? __ldg(p.s + j) : 0.f; };
+      float s_next = !PAGED && U.ntiles ? scale_of(key0) : 0.f;
       int next_vote = vote_interval(0) - 1;  // the same tile sequence in every warp
       // The warp's RW rows are NC chunks of 32 TMEM columns (chunk c at column
       // g * RW * H + 32 c, its head weights at ws_g + 32 c), taken in pairs; a
@@ -1189,8 +1220,16 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
       }
       for (int t = 0; t < U.ntiles; ++t, ++T) {
         const int j = key0 + t * kBlockKeys;
-        const float sj = s_next;
-        s_next = scale_of(j + kBlockKeys);  // (0 past the end)
+        float sj = s_next;
+        if (PAGED) {
+          // (read before this warp releases the tile's accumulator: the
+          // producer refills the entry only after every warp has done so)
+          const int e = static_cast<int>(T % SR);
+          if (!wait_phase<kSpin>(&sfull[e], (T / SR) & 1, abort_flag, p.status, limit)) aborted = true;
+          sj = j < U.len ? sring[e * kBlockKeys + qd * 32 + lane] : 0.f;
+        } else {
+          s_next = scale_of(j + kBlockKeys);  // (0 past the end)
+        }
         const uint32_t a = T & 1;
         // The last wait leaves the whole accumulator in registers: release it
         // to the MMA.  A row's logit sums its H / 32 chunks.  (fma with +0: an
@@ -1561,6 +1600,7 @@ __global__ void fill_empty_kernel(int32_t* out_idx, float* out_vals, int64_t tot
 template <int R, bool PAGED, int H, int MODE>
 static cudaError_t launch_indexer(const IndexerParams& p, int grid, cudaStream_t st) {
   static_assert(smem_layout<R, PAGED, H>().total + 1024 <= 227 * 1024, "shared memory per CTA");
+  static_assert(smem_layout<R, PAGED, H>().sring % 16 == 0, "bulk copies need 16-byte aligned destinations");
   const size_t smem = static_cast<size_t>(smem_layout<R, PAGED, H>().total) + 1024;
   auto kern = indexer_kernel<R, PAGED, H, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -26,7 +26,8 @@
  *     only enqueues work on it and returns.
  *   - Layouts are dense row-major: q [m, H, D], k [n, D], s [n], w [m, H],
  *     ks/ke [m], out [m, topk].
- *   - Alignment: q, k and k_pages 16 bytes (TMA); everything else 4 bytes;
+ *   - Alignment: q, k and k_pages 16 bytes (TMA), s_pages 16 bytes (bulk
+ *     copies of page scales); everything else 4 bytes;
  *     workspaces 256 bytes.
  *   - Errors are reported before anything is launched and leave the outputs
  *     untouched: FP8IDX_EINVAL (null pointer, misalignment, negative size,
