@@ -15,14 +15,15 @@ constexpr int kMaxTopK = 2048;
 constexpr int kPrefillRows = 8;    // query rows per prefill unit (row block)
 constexpr int kMaxEpiWarps = 12;   // epilogue warps per CTA at most (workspace scratch is sized for it)
 constexpr int kStatusBytes = 256;  // device status block at the head of every workspace
-// Tiles between two group votes of the fused epilogue, after t tiles of the
-// unit: short early, where the running threshold still moves fast, and
-// growing with the tiles already streamed (clamp(t / 4, min, max)), since the
-// threshold's relative movement per tile falls like 1 / t.
+// Tiles between two votes of an epilogue warp, after t tiles of the unit:
+// short early, where the running threshold still moves fast, and growing with
+// the tiles already streamed (clamp(t, min, max): the votes fall at about
+// t = 4, 8, 16, 32, then every 32 tiles), since the threshold's relative
+// movement per tile falls like 1 / t.
 constexpr int kMinVoteTiles = 4;
 constexpr int kMaxVoteTiles = 32;
 __host__ __device__ constexpr int vote_interval(int t) {
-  return t / 4 < kMinVoteTiles ? kMinVoteTiles : (t / 4 > kMaxVoteTiles ? kMaxVoteTiles : t / 4);
+  return t < kMinVoteTiles ? kMinVoteTiles : (t > kMaxVoteTiles ? kMaxVoteTiles : t);
 }
 
 // device status bits (workspace word 0)
