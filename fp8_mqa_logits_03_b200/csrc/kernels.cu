@@ -208,17 +208,17 @@ __device__ __forceinline__ Unit get_unit(const IndexerParams& p, int u) {
 // Bounded wait on an mbarrier phase.  Gives up when another role has
 // aborted or after `limit_ns`, flagging the device status; never traps.
 // NAP_NS == 0 polls with try_wait (for the epilogue's own hand-offs, where
-// the phase is normally complete already); NAP_NS > 0 tests the phase and
-// sleeps NAP_NS between tests, so that a role that is ahead of the epilogue
-// (MMA issue, TMA producer, idle select warps) takes few issue slots from it.
-// The abort flag and the clock are looked at every 8 polls.
+// the phase is normally complete already); NAP_NS > 0 passes try_wait a
+// suspend-time hint of 16 NAP_NS, so the thread sleeps in hardware until the
+// phase completes or the hint runs out, and a role that is ahead of the
+// epilogue (MMA issue, TMA producer, idle select warps) takes few issue
+// slots from it.  The abort flag and the clock are looked at every 8 tries.
 template <uint32_t NAP_NS>
 __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                        int* status, unsigned long long limit_ns) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (NAP_NS == 0 ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity)) return true;
-    if (NAP_NS) __nanosleep(NAP_NS);
+    if (NAP_NS == 0 ? mbar_try_wait(bar, parity) : mbar_try_wait_hint(bar, parity, 16 * NAP_NS)) return true;
     if ((it & 7) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > limit_ns) {
@@ -230,9 +230,10 @@ __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volatile 
   }
 }
 
-// Nap lengths (ns) by role: the epilogue polls; the MMA thread naps briefly
-// (it has slack against the epilogue but must not delay the next tile); the
-// producer runs stages ahead; idle roles sleep long.
+// Nap lengths (ns) by role, the unit of each role's suspend-time hint: the
+// epilogue polls; the MMA thread's is short (it has slack against the
+// epilogue but must not delay the next tile); the producer runs stages
+// ahead; idle roles sleep long.
 #ifndef FP8IDX_NAP_MMA_NS
 #define FP8IDX_NAP_MMA_NS 64
 #endif
