@@ -281,33 +281,63 @@ __device__ __forceinline__ uint32_t bar_red_popc(int id, int nthreads, bool pred
 }
 
 // sum_h w[h] * max(x[h], 0) over the 32 heads of one (key, row), for two
-// rows at once.  The max runs on the ALU pipe and the weighted sum as packed
-// two-lane FMAs (fma.rn.f32x2), so each head costs one ALU issue and half an
-// FMA issue.  Two packed accumulators per row (heads 4i, 4i+1 and 4i+2,
-// 4i+3) give four independent FMA chains; a packed add and one add join a
-// row's four partial sums.  Each operation rounds once.
+// rows at once.  Heads in groups of four; the first 8 - NABS groups take the
+// max on the ALU pipe and the weighted sum as packed two-lane FMAs
+// (fma.rn.f32x2): one ALU issue and half an FMA issue per head.  The last
+// NABS groups use 2 max(x, 0) = x + |x| instead, all on the FMA pipe (the
+// linear half packed, the |x| half with the free absolute-value operand
+// modifier), which moves work off the ALU pipe when it is the busier one.
+// Each operation rounds once.
+template <int NABS>
 __device__ __forceinline__ void relu_dot32_pair(const uint32_t (&xa)[32], const uint32_t (&xb)[32],
                                                 const float* wa, const float* wb, float& ra, float& rb) {
   const float4* wa4 = reinterpret_cast<const float4*>(wa);
   const float4* wb4 = reinterpret_cast<const float4*>(wb);
-  uint64_t la0 = 0, la1 = 0, lb0 = 0, lb1 = 0;
+  uint64_t la0 = 0, la1 = 0, lb0 = 0, lb1 = 0, ma0 = 0, mb0 = 0;
+  float aa0 = 0.f, aa1 = 0.f, ab0 = 0.f, ab1 = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 va = wa4[i], vb = wb4[i];
-    const float a0 = fmaxf(__uint_as_float(xa[4 * i + 0]), 0.f), a1 = fmaxf(__uint_as_float(xa[4 * i + 1]), 0.f);
-    const float a2 = fmaxf(__uint_as_float(xa[4 * i + 2]), 0.f), a3 = fmaxf(__uint_as_float(xa[4 * i + 3]), 0.f);
-    const float b0 = fmaxf(__uint_as_float(xb[4 * i + 0]), 0.f), b1 = fmaxf(__uint_as_float(xb[4 * i + 1]), 0.f);
-    const float b2 = fmaxf(__uint_as_float(xb[4 * i + 2]), 0.f), b3 = fmaxf(__uint_as_float(xb[4 * i + 3]), 0.f);
-    la0 = fma_f32x2(pack_f32x2(va.x, va.y), pack_f32x2(a0, a1), la0);
-    lb0 = fma_f32x2(pack_f32x2(vb.x, vb.y), pack_f32x2(b0, b1), lb0);
-    la1 = fma_f32x2(pack_f32x2(va.z, va.w), pack_f32x2(a2, a3), la1);
-    lb1 = fma_f32x2(pack_f32x2(vb.z, vb.w), pack_f32x2(b2, b3), lb1);
+    if (i < 8 - NABS) {
+      const float a0 = fmaxf(__uint_as_float(xa[4 * i + 0]), 0.f), a1 = fmaxf(__uint_as_float(xa[4 * i + 1]), 0.f);
+      const float a2 = fmaxf(__uint_as_float(xa[4 * i + 2]), 0.f), a3 = fmaxf(__uint_as_float(xa[4 * i + 3]), 0.f);
+      const float b0 = fmaxf(__uint_as_float(xb[4 * i + 0]), 0.f), b1 = fmaxf(__uint_as_float(xb[4 * i + 1]), 0.f);
+      const float b2 = fmaxf(__uint_as_float(xb[4 * i + 2]), 0.f), b3 = fmaxf(__uint_as_float(xb[4 * i + 3]), 0.f);
+      la0 = fma_f32x2(pack_f32x2(va.x, va.y), pack_f32x2(a0, a1), la0);
+      lb0 = fma_f32x2(pack_f32x2(vb.x, vb.y), pack_f32x2(b0, b1), lb0);
+      la1 = fma_f32x2(pack_f32x2(va.z, va.w), pack_f32x2(a2, a3), la1);
+      lb1 = fma_f32x2(pack_f32x2(vb.z, vb.w), pack_f32x2(b2, b3), lb1);
+    } else {
+      const float a0 = __uint_as_float(xa[4 * i + 0]), a1 = __uint_as_float(xa[4 * i + 1]);
+      const float a2 = __uint_as_float(xa[4 * i + 2]), a3 = __uint_as_float(xa[4 * i + 3]);
+      const float b0 = __uint_as_float(xb[4 * i + 0]), b1 = __uint_as_float(xb[4 * i + 1]);
+      const float b2 = __uint_as_float(xb[4 * i + 2]), b3 = __uint_as_float(xb[4 * i + 3]);
+      ma0 = fma_f32x2(pack_f32x2(va.x, va.y), pack_f32x2(a0, a1), ma0);
+      mb0 = fma_f32x2(pack_f32x2(vb.x, vb.y), pack_f32x2(b0, b1), mb0);
+      ma0 = fma_f32x2(pack_f32x2(va.z, va.w), pack_f32x2(a2, a3), ma0);
+      mb0 = fma_f32x2(pack_f32x2(vb.z, vb.w), pack_f32x2(b2, b3), mb0);
+      aa0 = fmaf(va.x, fabsf(a0), aa0);
+      ab0 = fmaf(vb.x, fabsf(b0), ab0);
+      aa1 = fmaf(va.y, fabsf(a1), aa1);
+      ab1 = fmaf(vb.y, fabsf(b1), ab1);
+      aa0 = fmaf(va.z, fabsf(a2), aa0);
+      ab0 = fmaf(vb.z, fabsf(b2), ab0);
+      aa1 = fmaf(va.w, fabsf(a3), aa1);
+      ab1 = fmaf(vb.w, fabsf(b3), ab1);
+    }
   }
   float p0, p1, q0, q1;
   unpack_f32x2(add_f32x2(la0, la1), p0, p1);
   unpack_f32x2(add_f32x2(lb0, lb1), q0, q1);
   ra = p0 + p1;
   rb = q0 + q1;
+  if (NABS > 0) {
+    float m0, m1, n0, n1;
+    unpack_f32x2(ma0, m0, m1);
+    unpack_f32x2(mb0, n0, n1);
+    ra += 0.5f * ((m0 + m1) + (aa0 + aa1));
+    rb += 0.5f * ((n0 + n1) + (ab0 + ab1));
+  }
 }
 
 // (Only meaningful for key >= base; any other key maps to some bin in range.)
@@ -1211,6 +1241,7 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
       // carry it from one iteration to the next); with two pairs the
       // registers this would hold across the filter are not there.
       constexpr bool kCarry = C::NC == 2;
+      constexpr int kAbsGroups = PAGED ? 0 : 2;  // head groups summed on the FMA pipe (see relu_dot32_pair)
       uint32_t xa[32], xb[32];
       if (kCarry && U.ntiles > 0) {
         if (!wait_phase<kSpin>(&tfull[T & 1], (T >> 1) & 1, abort_flag, p.status, limit)) aborted = true;
@@ -1250,17 +1281,17 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
             tc_fence_before();
             __syncwarp();
             mbar_arrive_if(lane == 0, &tempty[a]);
-            relu_dot32_pair(xa, xb, ws_g, ws_g + 32, Lc[0], Lc[1]);
+            relu_dot32_pair<kAbsGroups>(xa, xb, ws_g, ws_g + 32, Lc[0], Lc[1]);
           } else {
             uint32_t xc[32], xd[32];
             tmem_ld32(col0 + 64, xc);
             tmem_ld32(col0 + 96, xd);
-            relu_dot32_pair(xa, xb, ws_g, ws_g + 32, Lc[0], Lc[1]);
+            relu_dot32_pair<kAbsGroups>(xa, xb, ws_g, ws_g + 32, Lc[0], Lc[1]);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             mbar_arrive_if(lane == 0, &tempty[a]);
-            relu_dot32_pair(xc, xd, ws_g + 64, ws_g + 96, Lc[2], Lc[NC - 1]);
+            relu_dot32_pair<kAbsGroups>(xc, xd, ws_g + 64, ws_g + 96, Lc[2], Lc[NC - 1]);
           }
         }
         float L[RW];
