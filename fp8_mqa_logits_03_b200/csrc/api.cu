@@ -123,6 +123,8 @@ struct Plan {
   int H = 32;
   int n_chunks = 1;
   int chunk_keys = 0;
+  int tail_chunks = 0;  // the last tail_chunks chunks hold tail_keys keys each
+  int tail_keys = 0;
   int num_units = 0;
   int groups = 0;      // row blocks (prefill) or requests (paged)
   int64_t axis = 0;    // the whole key axis
@@ -196,6 +198,8 @@ int run_fused_topk(const Plan& pl, IndexerParams& p, uint8_t* wsb, bool paged, i
   const int topk = p.topk;
   p.n_chunks = pl.n_chunks;
   p.chunk_keys = pl.chunk_keys;
+  p.tail_chunks = pl.tail_chunks;
+  p.tail_keys = pl.tail_keys;
   p.num_units = pl.num_units;
   p.status = reinterpret_cast<int*>(wsb);
   p.cand = reinterpret_cast<uint2*>(wsb + pl.off_cand);
@@ -233,6 +237,7 @@ int run_fused_topk(const Plan& pl, IndexerParams& p, uint8_t* wsb, bool paged, i
   r.speculate = 0;
   r.n_chunks = 1;
   r.chunk_keys = static_cast<int>(round_up(std::max<int64_t>(pl.axis, 1), kBlockKeys));
+  r.tail_chunks = 0;
   r.num_units = pl.groups;
   r.cand = reinterpret_cast<uint2*>(wsb + pl.off_rcand);
   r.cand_cap = pl.rcap;
@@ -274,6 +279,7 @@ Plan plan_prefill(int64_t m, int64_t n, int topk, int sms, int H = kHeads) {
 // schedule; a unit's rows start from the thresholds their earlier chunks
 // raised, so later chunks pass few candidates.
 constexpr int kPagedUnitsPerSm = 8;
+constexpr int kPagedTailChunks = 4;
 Plan plan_paged(int64_t B, int R, int max_blocks, int topk, int sms, int H = kHeads) {
   Plan pl;
   pl.H = H;
@@ -287,6 +293,14 @@ Plan plan_paged(int64_t B, int R, int max_blocks, int topk, int sms, int H = kHe
     const int64_t ck = round_up(ceil_div(axis, want), kBlockKeys);
     pl.chunk_keys = static_cast<int>(ck);
     pl.n_chunks = static_cast<int>(ceil_div(axis, ck));
+    // the last kPagedTailChunks chunks each become two of half the size
+    const int m = std::min<int>(kPagedTailChunks, pl.n_chunks / 4);
+    const int64_t half = round_up(ceil_div(ck, 2), kBlockKeys);
+    if (m > 0 && half < ck) {
+      pl.tail_chunks = 2 * m;
+      pl.tail_keys = static_cast<int>(half);
+      pl.n_chunks += m;
+    }
   }
   finish_plan(pl, B, sms, topk, axis);
   return pl;

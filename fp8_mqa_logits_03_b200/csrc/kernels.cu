@@ -197,8 +197,12 @@ __device__ __forceinline__ Unit get_unit(const IndexerParams& p, int u) {
     lo = 0;
     hi = U.len;
   }
-  U.cbeg = c * p.chunk_keys;
-  U.cend = min(U.cbeg + p.chunk_keys, axis);
+  // chunks of chunk_keys keys, the last tail_chunks of them shorter (tail_keys):
+  // the chunk-major order claims those last, so the schedule ends on small units
+  const int nfull = p.n_chunks - p.tail_chunks;
+  const int clen = c < nfull ? p.chunk_keys : p.tail_keys;
+  U.cbeg = c < nfull ? c * p.chunk_keys : nfull * p.chunk_keys + (c - nfull) * p.tail_keys;
+  U.cend = min(U.cbeg + clen, axis);
   const int jb = max(U.cbeg, lo), je = min(U.cend, hi);
   U.jbeg = jb;
   U.ntiles = je > jb ? (je - jb + kBlockKeys - 1) / kBlockKeys : 0;

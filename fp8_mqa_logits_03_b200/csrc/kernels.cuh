@@ -61,6 +61,8 @@ struct IndexerParams {
   int rows_per_unit;  // query rows of a row block / request (at most the kernel's row capacity)
   int n_chunks;     // key chunks per row block / request
   int chunk_keys;   // keys per chunk (multiple of 128)
+  int tail_chunks;  // the last tail_chunks chunks hold tail_keys keys each (multiple of 128), the others chunk_keys
+  int tail_keys;
   int num_units;    // row blocks (or requests) x n_chunks
   // logits mode
   float* logits;
