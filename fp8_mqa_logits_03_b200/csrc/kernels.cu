@@ -872,6 +872,9 @@ __global__ void __launch_bounds__(Cfg<R, PAGED, H>::THREADS, 1) indexer_kernel(c
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // launched as a dependent grid, wait here for the grids before it on the
+  // stream to complete (a no-op otherwise)
+  griddep_wait();
   // a repair launch with nothing listed ends at once (the count is final: the
   // launches that list groups ran before this one on the stream)
   if (p.repair_mode && ld_volatile_i32(p.status + kRepairCount) == 0) return;
@@ -1511,6 +1514,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(const MergePara
   __shared__ int pre[kMergeMaxChunks + 1];
   __shared__ int wsum[kMergeWarps];
   extern __shared__ uint2 stage[];  // kMergeStage pairs (dynamic)
+  griddep_wait();  // the indexer's partial lists are complete
   const int row = blockIdx.x;
   const int unit_row = row / p.R;  // row block / request
   const int rl = row - unit_row * p.R;
@@ -1633,6 +1637,25 @@ __global__ void fill_empty_kernel(int32_t* out_idx, float* out_vals, int64_t tot
 
 // ------------------------------------------------------------------ launchers
 
+// Launch `kern`; `dependent`: as a programmatic dependent of the kernel before
+// it on the stream, which lets the launch overlap that kernel's end (the
+// kernel itself waits for it in griddep_wait before reading its results).
+template <class Kern, class Params>
+static cudaError_t launch_kernel(Kern kern, int grid, int block, size_t smem, cudaStream_t st, bool dependent,
+                                 const Params& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 template <int R, bool PAGED, int H, int MODE>
 static cudaError_t launch_indexer(const IndexerParams& p, int grid, cudaStream_t st) {
   static_assert(smem_layout<R, PAGED, H>().total + 1024 <= 227 * 1024, "shared memory per CTA");
@@ -1642,8 +1665,9 @@ static cudaError_t launch_indexer(const IndexerParams& p, int grid, cudaStream_t
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, Cfg<R, PAGED, H>::THREADS, smem, st>>>(p);
-  return cudaGetLastError();
+  // the repair launch follows a kernel of the same call on the stream: launch
+  // it as a dependent grid, so that its launch overlaps that kernel's end
+  return launch_kernel(kern, grid, Cfg<R, PAGED, H>::THREADS, smem, st, p.repair_mode != 0, p);
 }
 
 // Instantiations: 32 heads with 8-row prefill units (4- or 8-row paged
@@ -1666,8 +1690,7 @@ cudaError_t launch_merge(const MergeParams& p, cudaStream_t st) {
   constexpr int smem = kMergeStage * static_cast<int>(sizeof(uint2));
   cudaError_t e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  merge_kernel<<<p.rows, kMergeWarps * 32, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_kernel(merge_kernel, p.rows, kMergeWarps * 32, smem, st, true, p);  // (after the indexer)
 }
 
 cudaError_t launch_topk_rows(const TopkRowsParams& p, cudaStream_t st) {

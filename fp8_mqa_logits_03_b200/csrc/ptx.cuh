@@ -137,6 +137,11 @@ __device__ __forceinline__ void st_global_v2_if(bool pred, void* p, uint32_t a, 
       "l"(reinterpret_cast<uint64_t>(p)), "r"(a), "r"(b));
 }
 
+// Wait until the grids this one depends on (launched before it on the stream)
+// have completed and their memory is visible; a no-op in a grid launched
+// without programmatic stream serialisation.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
