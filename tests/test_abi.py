@@ -64,11 +64,11 @@ def test_logits_and_topk_rows_reject(L):
     assert L.fp8idx_topk_rows(FAKE, 10, FAKE, FAKE, 0, 10, 16, FAKE, None) == fx.OK
 
 
-def test_paged_rejects(L):
-    def call(R=4, page_size=64, H=32, B=2, max_blocks=4, num_pages=8, topk=64, q=FAKE):
-        return L.fp8idx_paged_mqa_logits_topk(q, FAKE, FAKE, FAKE, FAKE, FAKE, B, R, max_blocks,
-                                              num_pages, page_size, H, 128, topk, FAKE, None, FAKE,
-                                              1 << 20, None)
+@pytest.mark.parametrize("entry", ["fp8idx_paged_mqa_logits_topk", "fp8idx_paged_mqa_logits_topk_slots"])
+def test_paged_rejects(L, entry):
+    def call(R=4, page_size=64, H=32, B=2, max_blocks=4, num_pages=8, topk=64, q=FAKE, s_pages=FAKE):
+        return getattr(L, entry)(q, FAKE, s_pages, FAKE, FAKE, FAKE, B, R, max_blocks,
+                                 num_pages, page_size, H, 128, topk, FAKE, None, FAKE, 1 << 20, None)
     assert call(R=0) == fx.EUNSUPPORTED
     assert call(R=9) == fx.EUNSUPPORTED
     assert call(page_size=32) == fx.EUNSUPPORTED
@@ -76,6 +76,8 @@ def test_paged_rejects(L):
     assert call(H=64, R=5) == fx.EUNSUPPORTED    # 64 heads: at most 4 rows per request
     assert call(max_blocks=0) == fx.EINVAL
     assert call(q=MIS) == fx.EINVAL
+    assert call(s_pages=MIS) == fx.EINVAL        # page scales are bulk-copied: 16-byte aligned
+    assert b"16-byte" in L.fp8idx_last_error()
     assert call(B=0) == fx.OK
 
 
