@@ -491,9 +491,11 @@ SUITE = [(0, "fused"), (2, "fused"), (3, "fused"), (4, "fused"), (4, "act_quant"
 INDEX_PREP = [("decode", 1, 1.77), ("mtp4", 4, 1.81), ("prefill16", 16, 3.63)]
 
 
-def time_graph(call, reps_target_ms=200.0, samples=3):
-    """Median over `samples` of the mean replay time (us) of a CUDA graph of
-    `call`, each sample replaying for about reps_target_ms."""
+def time_graph(call, reps_target_ms=200.0, samples=3, per_graph=20):
+    """Median over `samples` of the mean time (us) of one `call`, from replays
+    of a CUDA graph holding `per_graph` calls back to back (so the graph's own
+    launch cost is spread over them), each sample replaying for about
+    reps_target_ms."""
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
@@ -503,7 +505,8 @@ def time_graph(call, reps_target_ms=200.0, samples=3):
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        call()
+        for _ in range(per_graph):
+            call()
     g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -521,7 +524,7 @@ def time_graph(call, reps_target_ms=200.0, samples=3):
             g.replay()
         e1.record()
         e1.synchronize()
-        out.append(e0.elapsed_time(e1) / reps * 1e3)
+        out.append(e0.elapsed_time(e1) / reps / per_graph * 1e3)
     del g
     return statistics.median(out)
 

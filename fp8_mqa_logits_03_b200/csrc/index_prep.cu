@@ -130,23 +130,45 @@ __global__ void __launch_bounds__(kPrepThreads)
   }
 }
 
-// (idx and out may be one buffer: each element is read, then written, by one thread)
-__global__ void transform_kernel(const int32_t* idx, int64_t rows, int topk,
-                                 const int32_t* __restrict__ row_base, const int32_t* __restrict__ row_table,
-                                 int rows_per_table_row, const int32_t* __restrict__ table, int64_t table_rows,
-                                 int64_t ld, int page_size, int32_t* out) {
-  const int64_t total = rows * topk;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t i = e / topk;
+// One CTA per (row, run of 256 positions): the row comes from the grid, not
+// from a division per element.  (idx and out may be one buffer: each element
+// is read, then written, by one thread.)
+constexpr int kTransformThreads = 256;
+
+__global__ void __launch_bounds__(kTransformThreads)
+    transform_kernel(const int32_t* idx, int64_t rows, int topk, const int32_t* __restrict__ row_base,
+                     const int32_t* __restrict__ row_table, int rows_per_table_row,
+                     const int32_t* __restrict__ table, int64_t table_rows, int64_t ld, int page_size,
+                     int page_shift, int32_t* out) {
+  const int x = static_cast<int>(blockIdx.x) * kTransformThreads + static_cast<int>(threadIdx.x);
+  if (x >= topk) return;
+  for (int64_t i = blockIdx.y; i < rows; i += gridDim.y) {
+    const int64_t e = i * topk + x;
     const int32_t v = idx[e];
     int32_t slot = -1;
     if (v >= 0) {
       const int64_t p = static_cast<int64_t>(v) - (row_base ? __ldg(row_base + i) : 0);
       const int64_t trow = row_table ? __ldg(row_table + i) : i / rows_per_table_row;
-      if (p >= 0 && trow >= 0 && trow < table_rows && p / page_size < ld) {
-        const int32_t page = __ldg(table + trow * ld + p / page_size);
-        if (page >= 0) slot = page * page_size + static_cast<int32_t>(p % page_size);
+      if (p >= 0 && trow >= 0 && trow < table_rows) {
+        // a power-of-two page size (1 or 64 in practice) takes a shift, and a
+        // position below 2^31 (always, unless the row base is negative) 32-bit
+        // arithmetic
+        int64_t blk, off;
+        if (page_shift >= 0) {
+          blk = p >> page_shift;
+          off = p & (page_size - 1);
+        } else if (p < (static_cast<int64_t>(1) << 31)) {
+          const int32_t b32 = static_cast<int32_t>(p) / page_size;
+          blk = b32;
+          off = p - static_cast<int64_t>(b32) * page_size;
+        } else {
+          blk = p / page_size;
+          off = p % page_size;
+        }
+        if (blk < ld) {
+          const int32_t page = __ldg(table + trow * ld + blk);
+          if (page >= 0) slot = page * page_size + static_cast<int32_t>(off);
+        }
       }
     }
     out[e] = slot;
@@ -176,11 +198,15 @@ cudaError_t launch_topk_transform(const int32_t* idx, int64_t rows, int topk, co
                                   const int32_t* row_table, int rows_per_table_row, const int32_t* table,
                                   int64_t table_rows, int64_t ld, int page_size, int32_t* out, int sms,
                                   cudaStream_t st) {
-  const int64_t total = rows * topk;
-  const int64_t want = (total + 255) / 256;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 8 * static_cast<int64_t>(sms))));
-  transform_kernel<<<grid, 256, 0, st>>>(idx, rows, topk, row_base, row_table, rows_per_table_row, table,
-                                         table_rows, ld, page_size, out);
+  if (rows <= 0 || topk <= 0) return cudaSuccess;
+  const unsigned gx = static_cast<unsigned>((topk + kTransformThreads - 1) / kTransformThreads);
+  // rows over grid y (at most 65535), each CTA looping over the rows it is given
+  const int64_t cap = std::max<int64_t>(1, std::min<int64_t>(65535, 16 * static_cast<int64_t>(sms)));
+  const unsigned gy = static_cast<unsigned>(std::min<int64_t>(rows, cap));
+  const int page_shift = (page_size & (page_size - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(page_size)) : -1;
+  transform_kernel<<<dim3(gx, gy), kTransformThreads, 0, st>>>(idx, rows, topk, row_base, row_table,
+                                                               rows_per_table_row, table, table_rows, ld,
+                                                               page_size, page_shift, out);
   return cudaGetLastError();
 }
 
