@@ -371,7 +371,7 @@ def make_case(fx, index, dev, path="fused"):
                     fx.mqa_logits(dv["q"][r0:r1], dv["k"], dv["s"], dv["w"][r0:r1], dv["ks"][r0:r1],
                                   dv["ke"][r0:r1], logits=lg)
                     fx.topk_rows(lg, dv["ks"][r0:r1], dv["ke"][r0:r1], topk, out=out[r0:r1])
-            kernel = (f"indexer_kernel<8,false,0> (materialised logits) + topk_rows_kernel, "
+            kernel = (f"indexer_kernel<8,false,32,0> (materialised logits) + topk_rows_kernel, "
                       f"{len(chunks)} row chunk(s) of <= {rows} rows")
             ws = None
             launches = 2 * len(chunks)
